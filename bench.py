@@ -1,0 +1,595 @@
+"""Benchmark: MoE token dispatch / combine on B200, one JSON line on rank 0.
+
+A step is one pass of the hot path over one batch: ep_layout (histogram,
+padded offsets, stable positions) -> ep_dispatch (FP8 E4M3 1x128 for the
+prefill and decode workloads, bf16 otherwise) -> ep_combine (fp32 fma, bf16
+out). The balanced workload adds ep_plan_balanced and ep_prefetch_weights.
+Inputs are seeded synthetic tensors resident in HBM before timing starts;
+every workload's inputs are larger than L2, so no flush runs between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the CPU oracle on a bounded sample
+
+value = algorithmic bytes of all steps on all ranks / max-over-ranks time.
+With N > 1 (torchrun, one process per GPU) every rank runs an independent
+replica of the workload on its own batch: the path has no exchange between
+logical ranks on one GPU, so the scaling is weak.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = ("dispatch/combine GB/s and µs per call on 1 B200; "
+          "fraction of HBM peak")
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+
+
+# --------------------------------------------------------------------------
+# byte accounting (algorithmic bytes: each input read once, each output
+# written once)
+# --------------------------------------------------------------------------
+
+def bytes_layout(N, K, E, used_rows):
+    # topk read by the histogram and by the position scan, pos written,
+    # row_src written over the used rows, counts / offsets
+    return 2 * N * K * 4 + N * K * 4 + used_rows * 4 + (2 * E + 1) * 4
+
+
+def bytes_dispatch(N, K, H, fp8, used_rows):
+    rd = N * H * 2 + N * K * 4 * 2 + used_rows * 4   # hidden, pos, w, row_src
+    if fp8:
+        wr = used_rows * (H + (H // 128) * 4 + 4)      # codes, scales, weight
+    else:
+        wr = used_rows * (H * 2 + 4)
+    return rd + wr
+
+
+def payload_dispatch(N, K, H, fp8):
+    """Bytes that land in the receive buffer for real tokens (the analogue
+    of the pages' per-link GB/s)."""
+    return N * K * (H + (H // 128) * 4 if fp8 else H * 2)
+
+
+def bytes_combine(N, K, H):
+    return N * K * H * 2 + N * K * 4 * 2 + N * H * 2
+
+
+def bytes_prefetch(n_slots, H, I):
+    return 3 * n_slots * H * I * 2 * 2
+
+
+# --------------------------------------------------------------------------
+# environment helpers
+# --------------------------------------------------------------------------
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def dist_info():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML every 10 ms."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting",
+        0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x10: "sync_boost",
+        0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            h = None
+            try:
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                h = pynvml.nvmlDeviceGetHandleByUUID(
+                    uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.h = h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(
+                h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(
+                    self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(
+                    nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit
+                 and n != "gpu_idle"]
+        return {"sm_mhz": (statistics.median(self.samples)
+                           if self.samples else None),
+                "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples), "source": "nvml"}
+
+
+def traffic_from_profiles(kernel: str, workload: str, src_file: str):
+    """DRAM bytes per launch recorded by ncu, if the profile summary names
+    the current source of the kernel (else None)."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    sha = hashlib.sha256(open(src_file, "rb").read()).hexdigest()[:16]
+    for line in open(p):
+        if line.startswith("#") or not line.strip():
+            continue
+        f = dict(kv.split("=", 1) for kv in line.split())
+        if (f.get("kernel") == kernel and f.get("workload") == workload
+                and f.get("src_sha") == sha):
+            return float(f["dram_bytes_per_launch"])
+    return None
+
+
+# --------------------------------------------------------------------------
+# the GPU path
+# --------------------------------------------------------------------------
+
+class Path:
+    """All device buffers of one replica, allocated once."""
+
+    def __init__(self, wl, dev, seed_offset=0):
+        import combine_ep_layout_09_b200 as ep
+        self.ep = ep
+        self.wl = wl
+        self.dev = dev
+        topk, w = workloads.routing(workloads.scaled(
+            wl, seed=wl.seed + seed_offset))
+        self.topk_np, self.w_np = topk, w
+        i32 = dict(dtype=torch.int32, device=dev)
+        self.topk = torch.from_numpy(topk).to(dev)
+        self.w = torch.from_numpy(w).to(dev)
+        self.hidden = workloads.bf16_normal((wl.N, wl.H), 1000 + wl.seed +
+                                            seed_offset, device=dev)
+        self.cap = ep.ep_capacity_bound(wl.N, wl.K, wl.E, wl.pad)
+        self.counts = torch.zeros(wl.E, **i32)
+        self.offsets = torch.zeros(wl.E + 1, **i32)
+        self.pos = torch.zeros(wl.N, wl.K, **i32)
+        self.row_src = torch.zeros(self.cap, **i32)
+        self.ws = torch.zeros(ep.ep_layout_workspace_bytes(wl.N, wl.K, wl.E),
+                              dtype=torch.uint8, device=dev)
+        self.status = torch.zeros(4, **i32)
+        if wl.fp8:
+            self.recv = torch.empty(self.cap, wl.H, dtype=torch.float8_e4m3fn,
+                                    device=dev)
+            self.scales = torch.empty(self.cap, wl.H // 128,
+                                      dtype=torch.float32, device=dev)
+        else:
+            self.recv = torch.empty(self.cap, wl.H, dtype=torch.bfloat16,
+                                    device=dev)
+            self.scales = None
+        self.recv_w = torch.empty(self.cap, dtype=torch.float32, device=dev)
+        # stand-in expert outputs, one bf16 row per receive row
+        self.y = workloads.expert_outputs(self.cap, wl.H, wl.seed +
+                                          seed_offset, device=dev)
+        self.out = torch.empty(wl.N, wl.H, dtype=torch.bfloat16, device=dev)
+        if wl.B > 0:
+            R, E, B = wl.R, wl.E, wl.B
+            self.plan = dict(cu=torch.empty(R, E + 1, **i32),
+                             expert=torch.empty(R, E, **i32),
+                             wrow=torch.empty(R, E, **i32),
+                             nseg=torch.empty(R, **i32),
+                             slot=torch.empty(R, B, **i32))
+            rows = E + R * B
+            self.W = [workloads.weight_buffer(rows, wl.H, wl.I, wl.seed + j,
+                                              device=dev) for j in range(3)]
+        self.launches_per_step = 4 + (2 if wl.B > 0 else 0)
+
+    def layout(self):
+        wl = self.wl
+        self.ep.ep_layout(self.topk, wl.R, wl.S, wl.K, wl.E, wl.pad,
+                          self.counts, self.offsets, self.pos, self.row_src,
+                          self.ws, self.status, cap=self.cap)
+
+    def plan_prefetch(self):
+        wl, p = self.wl, self.plan
+        self.ep.ep_plan_balanced(self.counts, wl.R, wl.S, wl.K, wl.E, wl.B,
+                                 p["cu"], p["expert"], p["wrow"], p["nseg"],
+                                 p["slot"], self.status)
+        self.ep.ep_prefetch_weights(p["slot"], wl.R, wl.E, wl.B, *self.W)
+
+    def dispatch(self):
+        wl = self.wl
+        self.ep.ep_dispatch(self.hidden, self.w, self.pos, self.row_src,
+                            self.offsets, wl.N, wl.K, wl.E, wl.H, wl.fp8,
+                            self.recv, self.scales, self.recv_w,
+                            status=self.status, cap=self.cap)
+
+    def combine(self):
+        wl = self.wl
+        self.ep.ep_combine(self.y, self.pos, self.w, wl.N, wl.K, wl.H,
+                           self.out, status=self.status, cap=self.cap)
+
+    def step(self, ev=None):
+        if ev is not None:
+            ev[0].record()
+        self.layout()
+        if ev is not None:
+            ev[1].record()
+        if self.wl.B > 0:
+            self.plan_prefetch()
+        if ev is not None:
+            ev[2].record()
+        self.dispatch()
+        if ev is not None:
+            ev[3].record()
+        self.combine()
+        if ev is not None:
+            ev[4].record()
+
+
+def run_gpu(args, wl):
+    ws, rank, local = dist_info()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(
+            seconds=120), device_id=dev)
+
+    def barrier():
+        if ws > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if ws == 1:
+            return x
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    path = Path(wl, dev, seed_offset=rank)
+    torch.cuda.synchronize()
+    # warm-up (also settles the used-row count for byte accounting)
+    for _ in range(args.warmup):
+        path.step()
+    torch.cuda.synchronize()
+    st = int(path.status[0].item())
+    if st:
+        raise RuntimeError(f"device status after warm-up: {st}")
+    used = int(path.offsets[-1].item())
+    n_slots = int((path.plan["slot"] >= 0).sum().item()) if wl.B else 0
+
+    b_lay = bytes_layout(wl.N, wl.K, wl.E, used)
+    b_dis = bytes_dispatch(wl.N, wl.K, wl.H, wl.fp8, used)
+    b_com = bytes_combine(wl.N, wl.K, wl.H)
+    b_pre = bytes_prefetch(n_slots, wl.H, wl.I) if wl.B else 0
+    b_step = b_lay + b_dis + b_com + b_pre
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)]
+           for _ in range(K)]
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record()
+        for i in range(K):
+            path.step(evs[i])
+        stop.record()
+        torch.cuda.synchronize()
+    barrier()
+    ms = start.elapsed_time(stop)
+    ms_max = max_over_ranks(ms)
+    per = {"layout": [], "plan_prefetch": [], "dispatch": [], "combine": []}
+    for e in evs:
+        per["layout"].append(e[0].elapsed_time(e[1]))
+        per["plan_prefetch"].append(e[1].elapsed_time(e[2]))
+        per["dispatch"].append(e[2].elapsed_time(e[3]))
+        per["combine"].append(e[3].elapsed_time(e[4]))
+    med = {k: statistics.median(v) * 1e3 for k, v in per.items()}   # us
+    avg = {k: statistics.fmean(v) * 1e3 for k, v in per.items()}
+    st = int(path.status[0].item())
+    if st:
+        raise RuntimeError(f"device status after timing: {st}")
+
+    # ---- end to end: host buffers in, host result out, every step -------
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, path, b_step, max_over_ranks, barrier)
+
+    result = None
+    if rank == 0:
+        peak, peak_src = measured_peak()
+        value = b_step * K * ws / (ms_max * 1e-3) / 1e9
+        comb_gbs = b_com / (avg["combine"] * 1e-6) / 1e9
+        dis_gbs = b_dis / (avg["dispatch"] * 1e-6) / 1e9
+        dom = "combine" if avg["combine"] >= avg["dispatch"] else "dispatch"
+        dom_bytes = b_com if dom == "combine" else b_dis
+        dom_gbs = comb_gbs if dom == "combine" else dis_gbs
+        kern = {"combine": ("k_combine", "combine.cu"),
+                "dispatch": ("k_dispatch", "dispatch.cu")}[dom]
+        src = os.path.join(ROOT, "combine_ep_layout_09_b200", "csrc", kern[1])
+        traffic = traffic_from_profiles(kern[0], wl.name, src)
+        clocks = clk.summary()
+        result = {
+            "metric": METRIC,
+            "value": round(value, 1),
+            "unit": "GB/s",
+            "n_gpus": ws,
+            "steps": K,
+            "warmup": args.warmup,
+            "ms_per_step": round(ms_max / K, 4),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic",
+            "config": {
+                "workload": wl.describe,
+                "step": ("ep_layout + " + ("ep_plan_balanced + "
+                         "ep_prefetch_weights + " if wl.B else "") +
+                         "ep_dispatch + ep_combine"),
+                "bytes_per_step": b_step,
+                "used_rows": used,
+                "l2": "no flush: every step moves >4 GB, inputs larger "
+                      "than the 126 MB L2",
+                "parallelism": f"{ws} independent replica(s), one per GPU",
+            },
+            "breakdown": {
+                "layout_us": round(med["layout"], 2),
+                "dispatch_us": round(med["dispatch"], 2),
+                "combine_us": round(med["combine"], 2),
+                "plan_prefetch_us": round(med["plan_prefetch"], 2),
+                "layout_plus_dispatch_us": round(med["layout"] +
+                                                 med["dispatch"], 2),
+                "dispatch_GBps": round(dis_gbs, 1),
+                "combine_GBps": round(comb_gbs, 1),
+                "dispatch_payload_GBps": round(
+                    payload_dispatch(wl.N, wl.K, wl.H, wl.fp8) /
+                    (avg["dispatch"] * 1e-6) / 1e9, 1),
+                "dispatch_bytes": b_dis, "combine_bytes": b_com,
+                "layout_bytes": b_lay, "prefetch_bytes": b_pre,
+                "frac_of_8TBps": {
+                    "dispatch": round(dis_gbs / NOMINAL_HBM_GBS, 4),
+                    "combine": round(comb_gbs / NOMINAL_HBM_GBS, 4)},
+                "frac_of_measured": {
+                    "dispatch": round(dis_gbs / peak, 4),
+                    "combine": round(comb_gbs / peak, 4)},
+            },
+            "roofline": {
+                "bound": "hbm",
+                "kernel": kern[0],
+                "achieved": round(dom_gbs, 1),
+                "peak": peak,
+                "unit": "GB/s",
+                "frac": round(dom_gbs / peak, 4),
+                "traffic": traffic,
+                "algorithmic_bytes": dom_bytes,
+                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_src == "measured" else "fallback 6.65 TB/s",
+            },
+            "clocks": clocks,
+            "e2e": e2e,
+            "gpu_launches": path.launches_per_step * K,
+            "gpu_launches_note": "kernels of libeplayout.so in the timed "
+                                 "region; ep_layout adds one cudaMemsetAsync "
+                                 "per step",
+        }
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def run_e2e(args, path, b_step, max_over_ranks, barrier):
+    """Same step with the user's inputs in pinned host memory: H2D of
+    hidden, topk and route weights, the three calls, D2H of the combined
+    output, all inside the timed region."""
+    wl = path.wl
+    h_hidden = path.hidden.cpu().pin_memory()
+    h_topk = path.topk.cpu().pin_memory()
+    h_w = path.w.cpu().pin_memory()
+    h_out = torch.empty(path.out.shape, dtype=path.out.dtype).pin_memory()
+    steps = max(1, min(args.steps, args.e2e_steps))
+
+    def one():
+        path.hidden.copy_(h_hidden, non_blocking=True)
+        path.topk.copy_(h_topk, non_blocking=True)
+        path.w.copy_(h_w, non_blocking=True)
+        path.step()
+        h_out.copy_(path.out, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for _ in range(steps):
+        one()
+    stop.record()
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(start.elapsed_time(stop))
+    ws, _, _ = dist_info()
+    h2d = (h_hidden.numel() * h_hidden.element_size() + h_topk.numel() * 4 +
+           h_w.numel() * 4)
+    d2h = h_out.numel() * h_out.element_size()
+    return {"value": round(b_step * steps * ws / (ms * 1e-3) / 1e9, 1),
+            "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(ms / steps, 3),
+            "note": "expert outputs (combine input) stay device-resident"}
+
+
+# --------------------------------------------------------------------------
+# the CPU oracle (baseline / reference arm)
+# --------------------------------------------------------------------------
+
+def oracle_sample(wl, n_tok, seed_offset=0):
+    """Inputs for the first n_tok tokens of the workload (host)."""
+    topk, w = workloads.routing(workloads.scaled(wl, seed=wl.seed +
+                                                 seed_offset))
+    hid = workloads.bf16_normal((n_tok, wl.H), 1000 + wl.seed + seed_offset)
+    h = hid.view(torch.int16).numpy().view(np.uint16)
+    y = workloads.expert_outputs(n_tok * wl.K, wl.H, wl.seed + seed_offset)
+    y = y.view(torch.int16).numpy().view(np.uint16)
+    return topk[:n_tok], w[:n_tok], h, y
+
+
+def time_oracle_step(wl, topk, w, h, y):
+    """One oracle pass over the sample: layout, dispatch, combine. Returns
+    (seconds, algorithmic bytes of the sample)."""
+    import oracle
+    n = topk.shape[0]
+    t0 = time.perf_counter()
+    lay = oracle.layout(topk, wl.E, wl.pad)
+    cap = int(lay["offsets"][-1])
+    if wl.fp8:
+        oracle.dispatch_fp8(h, w, lay, wl.E, max(cap, 1))
+    else:
+        oracle.dispatch_bf16(h, w, lay, wl.E, max(cap, 1))
+    pos = np.arange(n * wl.K, dtype=np.int32).reshape(n, wl.K)
+    oracle.combine(y, pos, w)
+    dt = time.perf_counter() - t0
+    b = (bytes_layout(n, wl.K, wl.E, cap) +
+         bytes_dispatch(n, wl.K, wl.H, wl.fp8, cap) +
+         bytes_combine(n, wl.K, wl.H))
+    return dt, b
+
+
+def cpu_baseline(wl, n_tok):
+    topk, w, h, y = oracle_sample(wl, n_tok)
+    dt, b = time_oracle_step(wl, topk, w, h, y)
+    return {"value": round(b / dt / 1e9, 3), "unit": "GB/s", "cores": 1,
+            "kind": "oracle", "seconds": round(dt, 2),
+            "sample": f"tokens 0..{n_tok - 1} of {wl.N}: layout, "
+                      f"{'FP8' if wl.fp8 else 'bf16'} dispatch and combine "
+                      "of the sample, single-threaded C"}
+
+
+def run_reference(args, wl):
+    ws, rank, _ = dist_info()
+    if rank != 0:
+        return None
+    # about a minute of oracle work for the whole warm-up + timed run
+    per_tok = 0.8e-3
+    n_tok = int(max(1, min(4096, 60.0 / (args.steps + args.warmup) /
+                           per_tok)))
+    topk, w, h, y = oracle_sample(wl, n_tok)
+    for _ in range(args.warmup):
+        time_oracle_step(wl, topk, w, h, y)
+    tot_t, tot_b = 0.0, 0
+    for _ in range(args.steps):
+        dt, b = time_oracle_step(wl, topk, w, h, y)
+        tot_t += dt
+        tot_b += b
+    value = tot_b / tot_t / 1e9
+    sample = (f"each step: tokens 0..{n_tok - 1} of {wl.N}: layout, "
+              f"{'FP8' if wl.fp8 else 'bf16'} dispatch and combine of the "
+              "sample, single-threaded C oracle")
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 3), "unit": "GB/s",
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(tot_t / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl.describe,
+                   "step": "oracle layout + dispatch + combine"},
+        "cpu_baseline": {"value": round(value, 3), "unit": "GB/s",
+                         "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "GB/s",
+                "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="prefill",
+                    choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=8192)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = workloads.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        res = run_reference(args, wl)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    res = run_gpu(args, wl)
+    ws, rank, _ = dist_info()
+    if rank == 0:
+        if ws == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(
+                wl, min(wl.N, args.cpu_sample_tokens))
+        else:
+            res["cpu_baseline"] = None
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,202 @@
+// api.cu -- the extern "C" entry points of libeplayout.so (include/eplayout.h):
+// argument validation on the host, then the kernel launchers.
+#include <climits>
+#include <cstdint>
+
+#include "../../include/eplayout.h"
+#include "ep_launch.h"
+
+namespace {
+
+constexpr int kAbiVersion = 1;
+constexpr int kMaxK = 32;
+constexpr int kMaxH = 32768;
+constexpr int64_t kMaxEntries = (int64_t(1) << 30) - 1;
+
+bool aligned16(const void* p) {
+  return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+bool status_ok(const int32_t* s) {
+  return s == nullptr || (reinterpret_cast<uintptr_t>(s) & 3u) == 0;
+}
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+int sms_or_all(int num_sms) {
+  const int all = ep::device_sm_count();
+  if (num_sms <= 0 || num_sms > all) return all;
+  return num_sms;
+}
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? EP_OK : EP_ERR_CUDA; }
+
+}  // namespace
+
+namespace ep {
+
+int device_sm_count() {
+  static int cache[128] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) !=
+            cudaSuccess ||
+        n <= 0)
+      return 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+}  // namespace ep
+
+extern "C" {
+
+int ep_abi_version(void) { return kAbiVersion; }
+
+const char* ep_strerror(int code) {
+  switch (code) {
+    case EP_OK: return "ok";
+    case EP_ERR_INVALID_ARG: return "invalid argument";
+    case EP_ERR_ALIGNMENT: return "pointer NULL or not 16-byte aligned";
+    case EP_ERR_WORKSPACE: return "workspace too small";
+    case EP_ERR_CAPACITY: return "capacity below the static bound or above INT32_MAX";
+    case EP_ERR_CUDA: return "CUDA launch failed";
+    case EP_DEV_BAD_EXPERT: return "device: expert id outside [0, E)";
+    case EP_DEV_CAPACITY: return "device: row index outside [0, cap)";
+    case EP_DEV_TIMEOUT: return "device: bounded wait gave up";
+    case EP_DEV_SLOTS: return "device: balanced plan ran out of prefetch slots";
+    case EP_DEV_PLAN_TOTAL: return "device: tokens_per_expert does not sum to R*S*K";
+    default: return "unknown code";
+  }
+}
+
+int64_t ep_capacity_bound(int64_t num_tokens, int K, int E, int token_padding) {
+  if (num_tokens < 0 || K < 1 || E < 1 || token_padding < 1) return -1;
+  return num_tokens * K + int64_t(E) * (token_padding - 1);
+}
+
+size_t ep_layout_workspace_bytes(int64_t num_tokens, int K, int E) {
+  if (num_tokens < 0 || K < 1 || K > kMaxK || E < 1 || E > ep::kMaxExperts)
+    return 0;
+  return ep::layout_workspace_bytes(num_tokens * K, E);
+}
+
+int ep_layout(const int32_t* topk_experts, int R, int S, int K, int E,
+              int token_padding, int32_t* tokens_per_expert,
+              int32_t* expert_offsets, int32_t* pos, int32_t* row_src,
+              int64_t cap, void* workspace, size_t workspace_bytes,
+              int32_t* status, void* stream) {
+  if (R < 1 || S < 0 || K < 1 || K > kMaxK || E < 1 || E > ep::kMaxExperts ||
+      E % R != 0 || token_padding < 1)
+    return EP_ERR_INVALID_ARG;
+  const int64_t N = int64_t(R) * S;
+  const int64_t M = N * K;
+  if (M > kMaxEntries) return EP_ERR_INVALID_ARG;
+  const int64_t bound = ep_capacity_bound(N, K, E, token_padding);
+  if (cap < bound || cap > INT32_MAX) return EP_ERR_CAPACITY;
+  if (!aligned16(tokens_per_expert) || !aligned16(expert_offsets) ||
+      !aligned16(workspace) || !status_ok(status))
+    return EP_ERR_ALIGNMENT;
+  if (M > 0 && (!aligned16(topk_experts) || !aligned16(pos)))
+    return EP_ERR_ALIGNMENT;
+  if (cap > 0 && !aligned16(row_src)) return EP_ERR_ALIGNMENT;
+  if (workspace_bytes < ep::layout_workspace_bytes(M, E)) return EP_ERR_WORKSPACE;
+  return cuda_rc(ep::launch_layout(topk_experts, M, E, token_padding,
+                                   tokens_per_expert, expert_offsets, pos,
+                                   row_src, cap, workspace, status,
+                                   sms_or_all(0), as_stream(stream)));
+}
+
+int ep_dispatch(const void* hidden, const float* route_weights,
+                const int32_t* pos, const int32_t* row_src,
+                const int32_t* expert_offsets, int64_t num_tokens, int K,
+                int E, int H, int64_t cap, int fp8, void* recv,
+                float* recv_scales, float* recv_weights, int num_sms,
+                int32_t* status, void* stream) {
+  if (num_tokens < 0 || K < 1 || K > kMaxK || E < 1 || H < 8 || H > kMaxH ||
+      H % 8 != 0 || (fp8 != 0 && fp8 != 1) || (fp8 && H % 128 != 0) ||
+      cap < 0 || cap > INT32_MAX || num_sms < 0 ||
+      num_tokens * K > kMaxEntries)
+    return EP_ERR_INVALID_ARG;
+  if (!aligned16(expert_offsets) || !status_ok(status)) return EP_ERR_ALIGNMENT;
+  if (num_tokens > 0 && (!aligned16(hidden) || !aligned16(route_weights) ||
+                         !aligned16(pos)))
+    return EP_ERR_ALIGNMENT;
+  if (cap > 0 && (!aligned16(row_src) || !aligned16(recv))) return EP_ERR_ALIGNMENT;
+  if (cap > 0 && fp8 && !aligned16(recv_scales)) return EP_ERR_ALIGNMENT;
+  if (recv_weights && !aligned16(recv_weights)) return EP_ERR_ALIGNMENT;
+  if (num_tokens == 0 && cap == 0) return EP_OK;
+  return cuda_rc(ep::launch_dispatch(hidden, route_weights, pos, row_src,
+                                     expert_offsets, num_tokens, K, E, H, cap,
+                                     fp8 != 0, recv, fp8 ? recv_scales : nullptr,
+                                     recv_weights, sms_or_all(num_sms), status,
+                                     as_stream(stream)));
+}
+
+int ep_combine(const void* expert_out, const int32_t* pos,
+               const float* route_weights, int64_t num_tokens, int K, int H,
+               int64_t cap, void* out, int num_sms, int32_t* status,
+               void* stream) {
+  if (num_tokens < 0 || K < 1 || K > kMaxK || H < 8 || H > kMaxH ||
+      H % 8 != 0 || cap < 0 || cap > INT32_MAX || num_sms < 0 ||
+      num_tokens * K > kMaxEntries)
+    return EP_ERR_INVALID_ARG;
+  if (!status_ok(status)) return EP_ERR_ALIGNMENT;
+  if (num_tokens == 0) return EP_OK;
+  if (!aligned16(pos) || !aligned16(route_weights) || !aligned16(out))
+    return EP_ERR_ALIGNMENT;
+  if (cap > 0 && !aligned16(expert_out)) return EP_ERR_ALIGNMENT;
+  return cuda_rc(ep::launch_combine(expert_out, pos, route_weights, num_tokens,
+                                    K, H, cap, out, sms_or_all(num_sms),
+                                    status, as_stream(stream)));
+}
+
+int ep_plan_balanced(const int32_t* tokens_per_expert, int R, int S, int K,
+                     int E, int B, int32_t* plan_cu, int32_t* plan_expert,
+                     int32_t* plan_wrow, int32_t* plan_nseg,
+                     int32_t* slot_expert, int32_t* status, void* stream) {
+  if (R < 1 || S < 0 || K < 1 || K > kMaxK || E < 1 || E > ep::kMaxExperts ||
+      B < 0 || int64_t(R) * S * K > kMaxEntries || int64_t(R) * B > INT32_MAX)
+    return EP_ERR_INVALID_ARG;
+  if (!aligned16(tokens_per_expert) || !aligned16(plan_cu) ||
+      !aligned16(plan_expert) || !aligned16(plan_wrow) || !aligned16(plan_nseg) ||
+      !status_ok(status))
+    return EP_ERR_ALIGNMENT;
+  if (B > 0 && !aligned16(slot_expert)) return EP_ERR_ALIGNMENT;
+  return cuda_rc(ep::launch_plan_balanced(tokens_per_expert, R, S, K, E, B,
+                                          plan_cu, plan_expert, plan_wrow,
+                                          plan_nseg, slot_expert, status,
+                                          as_stream(stream)));
+}
+
+int ep_prefetch_weights(const int32_t* slot_expert, int R, int E, int B,
+                        int64_t elems_per_expert, void* gate, void* up,
+                        void* down, int num_sms, void* stream) {
+  if (R < 1 || E < 1 || B < 0 || elems_per_expert < 0 ||
+      (elems_per_expert * 2) % 16 != 0 || num_sms < 0)
+    return EP_ERR_INVALID_ARG;
+  if (B == 0 || elems_per_expert == 0) return EP_OK;
+  if (!aligned16(slot_expert) || !aligned16(gate) || !aligned16(up) ||
+      !aligned16(down))
+    return EP_ERR_ALIGNMENT;
+  return cuda_rc(ep::launch_prefetch(slot_expert, R, E, B, elems_per_expert,
+                                     gate, up, down, sms_or_all(num_sms),
+                                     as_stream(stream)));
+}
+
+int ep_debug_e4m3_encode(const float* x, uint8_t* out, int64_t n,
+                         void* stream) {
+  if (n < 0) return EP_ERR_INVALID_ARG;
+  if (n == 0) return EP_OK;
+  if (!aligned16(x) || !aligned16(out)) return EP_ERR_ALIGNMENT;
+  return cuda_rc(ep::launch_debug_e4m3(x, out, n, as_stream(stream)));
+}
+
+int ep_debug_bounded_wait(const int32_t* flag, int64_t max_polls,
+                          int32_t* status, void* stream) {
+  if (max_polls < 0) return EP_ERR_INVALID_ARG;
+  if (!aligned16(flag) || status == nullptr || !status_ok(status))
+    return EP_ERR_ALIGNMENT;
+  return cuda_rc(ep::launch_debug_wait(flag, max_polls, status, as_stream(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,62 @@
+// ep_launch.h -- host-side launchers of the kernels, called by api.cu after
+// argument validation. Every launcher enqueues on `stream` and returns the
+// launch's cudaError_t.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace ep {
+
+// ---- layout ---------------------------------------------------------------
+
+// Entries handled by one CTA of the position scan (its look-back tile).
+constexpr int kScanTile = 4096;
+// Largest E the layout kernels keep in shared memory.
+constexpr int kMaxExperts = 1024;
+
+size_t layout_workspace_bytes(int64_t entries, int E);
+
+cudaError_t launch_layout(const int32_t* topk, int64_t entries, int E, int pad,
+                          int32_t* tokens_per_expert, int32_t* expert_offsets,
+                          int32_t* pos, int32_t* row_src, int64_t cap,
+                          void* workspace, int32_t* status, int num_sms,
+                          cudaStream_t stream);
+
+// ---- dispatch / combine ---------------------------------------------------
+
+cudaError_t launch_dispatch(const void* hidden, const float* w,
+                            const int32_t* pos, const int32_t* row_src,
+                            const int32_t* expert_offsets, int64_t N, int K,
+                            int E, int H, int64_t cap, bool fp8, void* recv,
+                            float* recv_scales, float* recv_w, int num_sms,
+                            int32_t* status, cudaStream_t stream);
+
+cudaError_t launch_combine(const void* y, const int32_t* pos, const float* w,
+                           int64_t N, int K, int H, int64_t cap, void* out,
+                           int num_sms, int32_t* status, cudaStream_t stream);
+
+// ---- balanced plan / prefetch ---------------------------------------------
+
+cudaError_t launch_plan_balanced(const int32_t* counts, int R, int S, int K,
+                                 int E, int B, int32_t* plan_cu,
+                                 int32_t* plan_expert, int32_t* plan_wrow,
+                                 int32_t* plan_nseg, int32_t* slot_expert,
+                                 int32_t* status, cudaStream_t stream);
+
+cudaError_t launch_prefetch(const int32_t* slot_expert, int R, int E, int B,
+                            int64_t elems, void* gate, void* up, void* down,
+                            int num_sms, cudaStream_t stream);
+
+// ---- diagnostics ----------------------------------------------------------
+
+cudaError_t launch_debug_e4m3(const float* x, uint8_t* out, int64_t n,
+                             cudaStream_t stream);
+cudaError_t launch_debug_wait(const int32_t* flag, int64_t max_polls,
+                              int32_t* status, cudaStream_t stream);
+
+// SM count of the current device (cached per device).
+int device_sm_count();
+
+}  // namespace ep

@@ -1,0 +1,239 @@
+/*
+ * eplayout.h -- C ABI of libeplayout.so: MoE token dispatch / combine with an
+ * expert-grouped receive layout, on one NVIDIA B200 (sm_100a).
+ *
+ * Expert-parallel ranks are logical: the receive regions of all R ranks live
+ * in one device buffer, rank-major, experts in order inside each rank
+ * ("Экспертный параллелизм (EP)" glossary, "Что подтверждено": E experts over
+ * ep_size ranks, E divisible by ep_size, E/ep_size local experts per rank;
+ * rank r owns experts [r*E/R, (r+1)*E/R)).
+ *
+ * Conventions shared by every entry point
+ *   - Every data pointer is a DEVICE pointer owned by the caller. The library
+ *     allocates no memory, never synchronises the device or the stream, and
+ *     enqueues all of its work on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream). Output buffers are fully overwritten over the ranges
+ *     stated below; nothing is read from them.
+ *   - Arrays are dense and row-major. bf16 is IEEE bfloat16, e4m3 is the OCP
+ *     FP8 E4M3 ("fn") format, weights are IEEE fp32.
+ *   - Token t of logical rank r has global index t = r*S + s. Entry (t,k) has
+ *     flat index t*K + k.
+ *   - Return value: EP_OK (0) or a negative EP_ERR_* code; on error nothing
+ *     has been enqueued. Arguments are checked on the host before any CUDA
+ *     call. Conditions only the device can see are OR-ed into `*status`, a
+ *     device int32 the caller zeroes beforehand and reads when it wishes
+ *     (EP_DEV_* bits). No kernel traps; every device-side wait is bounded.
+ *   - Every array pointer must be non-NULL and 16-byte aligned unless stated
+ *     otherwise; `status` may be NULL (no reporting) or 4-byte aligned
+ *     (EP_ERR_ALIGNMENT otherwise).
+ */
+#ifndef EPLAYOUT_H_
+#define EPLAYOUT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define EP_API __attribute__((visibility("default")))
+#else
+#define EP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* return codes */
+#define EP_OK 0
+#define EP_ERR_INVALID_ARG (-1) /* a size or flag outside its stated range */
+#define EP_ERR_ALIGNMENT (-2)   /* a pointer that is NULL or not 16-B aligned */
+#define EP_ERR_WORKSPACE (-3)   /* workspace smaller than ep_layout_workspace_bytes */
+#define EP_ERR_CAPACITY (-4)    /* cap below ep_capacity_bound, or above INT32_MAX */
+#define EP_ERR_CUDA (-5)        /* a CUDA launch or attribute call failed */
+
+/* device status bits (OR-ed into *status) */
+#define EP_DEV_BAD_EXPERT 1  /* an expert id outside [0, E); that entry skipped */
+#define EP_DEV_CAPACITY 2    /* a row index outside [0, cap); that access skipped */
+#define EP_DEV_TIMEOUT 4     /* a bounded device-side wait gave up */
+#define EP_DEV_SLOTS 8       /* the balanced plan needed more than B slots on a rank */
+#define EP_DEV_PLAN_TOTAL 16 /* sum(tokens_per_expert) != R*S*K; plan not written */
+
+/* Version of this ABI (bumped on any signature change). */
+EP_API int ep_abi_version(void);
+
+/* Static text for a return code or a single status bit. */
+EP_API const char* ep_strerror(int code);
+
+/* Rows any routing of N tokens can need once each expert's group is padded
+ * to a multiple of token_padding: N*K + E*(token_padding-1). Negative on
+ * invalid arguments. ("MoonEP核心功能深度剖析", "2. 高效通信机制": static
+ * shapes, so the receive buffer is sized without a host sync.) */
+EP_API int64_t ep_capacity_bound(int64_t num_tokens, int K, int E, int token_padding);
+
+/* Bytes of scratch ep_layout needs for N tokens, K, E (0 on invalid input). */
+EP_API size_t ep_layout_workspace_bytes(int64_t num_tokens, int K, int E);
+
+/*
+ * ep_layout -- steps 1-3 of dispatch: count tokens per expert, pad each
+ * expert's group, and give every (token, k) entry its final row in the
+ * expert-grouped receive buffer ("MoonEP核心功能深度剖析", "2. 高效通信机制":
+ * tokens are written straight to their final expert-grouped position;
+ * "快速上手": tokens_per_expert [E], token_padding; search results for
+ * "EP Moe": padding instead of dropping).
+ *
+ * in   topk_experts      int32 [N, K], N = R*S; ids in [0, E)
+ *      R, S, K, E        logical ranks, tokens per rank, experts per token,
+ *                        experts; E % R == 0, 1 <= K <= 32, 1 <= E <= 1024,
+ *                        N*K < 2^30
+ *      token_padding     >= 1; each expert's group is rounded up to a
+ *                        multiple of it
+ * out  tokens_per_expert int32 [E]
+ *      expert_offsets    int32 [E+1]: expert e owns rows
+ *                        [off[e], off[e+1]); off[E] = rows used; rank r's
+ *                        region is [off[r*E/R], off[(r+1)*E/R])
+ *      pos               int32 [N, K]: row of entry (t,k); -1 for a bad id.
+ *                        Inside an expert's group rows follow (t, k) order.
+ *      row_src           int32 [cap]: t*K+k for every used row, -1 for
+ *                        padding rows in [0, off[E]); rows >= off[E] untouched
+ *      cap               rows of row_src; ep_capacity_bound(...) <= cap
+ *                        <= INT32_MAX
+ *      workspace         scratch of >= ep_layout_workspace_bytes(N, K, E)
+ *                        bytes, contents ignored and overwritten; must not be
+ *                        shared by two calls in flight at the same time
+ *      status            device int32, EP_DEV_BAD_EXPERT / EP_DEV_TIMEOUT /
+ *                        EP_DEV_CAPACITY may be OR-ed in
+ * Three launches (one memset, two kernels) on `stream`.
+ */
+EP_API int ep_layout(const int32_t* topk_experts, int R, int S, int K, int E,
+              int token_padding, int32_t* tokens_per_expert,
+              int32_t* expert_offsets, int32_t* pos, int32_t* row_src,
+              int64_t cap, void* workspace, size_t workspace_bytes,
+              int32_t* status, void* stream);
+
+/*
+ * ep_dispatch -- step 4: copy every token row to its K receive rows
+ * ("Экспертный параллелизм (EP)", "Что подтверждено": token activations are
+ * sent to the experts; "DeepSeek开源周第二天：DeepEP深度分析", "性能": FP8
+ * dispatch; "MoonEP核心功能深度剖析", "快速上手": dispatch(hidden_sh,
+ * route_weights_sk, topk_experts_sk, ...) -> hidden_nvsh, route_weights_nvs).
+ *
+ * in   hidden            bf16 [N, H]
+ *      route_weights     fp32 [N, K]
+ *      pos, row_src,
+ *      expert_offsets    as written by ep_layout for the same topk
+ *      N, K, E, H        H % 8 == 0 (bf16), H % 128 == 0 (fp8), H <= 32768
+ *      cap               rows of recv / recv_scales / recv_weights
+ *      fp8               0: recv is bf16 [cap, H], a bit copy of the row.
+ *                        1: recv is e4m3 [cap, H]; per row and 128-channel
+ *                        group g: amax = max|x|, scale = amax / 448 (fp32,
+ *                        round to nearest), code = e4m3(x / scale) with the
+ *                        quotient in fp32 and the encoding round-to-nearest-
+ *                        even, saturating to +-448; scale 0 gives code 0.
+ * out  recv              rows pos[t,k] <- token t; padding rows (row_src ==
+ *                        -1 below off[E]) <- zeros; rows >= off[E] untouched
+ *      recv_scales       fp32 [cap, H/128] when fp8 (padding rows 0), else
+ *                        ignored (may be NULL)
+ *      recv_weights      fp32 [cap]: w[t,k] at pos[t,k], 0 on padding rows;
+ *                        may be NULL
+ *      num_sms           SMs to use, 0 = all
+ *      status            EP_DEV_CAPACITY, EP_DEV_TIMEOUT may be OR-ed in
+ */
+EP_API int ep_dispatch(const void* hidden, const float* route_weights,
+                const int32_t* pos, const int32_t* row_src,
+                const int32_t* expert_offsets, int64_t num_tokens, int K,
+                int E, int H, int64_t cap, int fp8, void* recv,
+                float* recv_scales, float* recv_weights, int num_sms,
+                int32_t* status, void* stream);
+
+/*
+ * ep_combine -- gather each token's K expert outputs and reduce them with the
+ * route weights, back in token order ("Экспертный параллелизм (EP)", "Что
+ * подтверждено": the results come back through a second AllToAll and are
+ * combined; "DeepSeek开源周第二天：DeepEP深度分析", "性能": BF16 combine;
+ * "MoonEP核心功能深度剖析", "快速上手": combine(plan, expert_output_nvsh, ...)
+ * -> output_sh).
+ *
+ * in   expert_out        bf16 [cap, H], row pos[t,k] holds expert output
+ *      pos               int32 [N, K] (entries < 0 are skipped)
+ *      route_weights     fp32 [N, K]
+ * out  out               bf16 [N, H]:
+ *                        out[t,h] = bf16_rne(acc), acc = +0 then for k = 0..K-1
+ *                        acc = fma(w[t,k], float(y[pos[t,k], h]), acc) in fp32
+ *      num_sms           SMs to use, 0 = all
+ *      status            EP_DEV_CAPACITY may be OR-ed in
+ */
+EP_API int ep_combine(const void* expert_out, const int32_t* pos,
+               const float* route_weights, int64_t num_tokens, int K, int H,
+               int64_t cap, void* out, int num_sms, int32_t* status,
+               void* stream);
+
+/*
+ * ep_plan_balanced -- the perfectly balanced plan ("MoonEP核心功能深度剖析",
+ * "1. 完美负载平衡": every rank receives exactly S*K rows however skewed the
+ * routing, through a few redundant experts planned online; "3. 智能内存管理":
+ * the weight buffer holds all experts in rows [0, E) and each rank's prefetch
+ * slots after them).
+ *
+ * The unpadded expert-grouped rows (ep_layout with token_padding = 1) are cut
+ * into R chunks of exactly T = S*K rows; chunk d is rank d's receive region.
+ * A segment is one expert's rows inside one chunk. The chunk holding an
+ * expert's first row reads its own weight row e; each later chunk the expert
+ * reaches takes that rank's next free slot b and weight row E + d*B + b.
+ *
+ * in   tokens_per_expert int32 [E], must sum to R*S*K
+ *      R, S, K, E, B     B = prefetch slots per rank (>= 0)
+ * out  plan_cu           int32 [R, E+1]: segment j of rank d covers chunk
+ *                        rows [cu[d,j], cu[d,j+1]); cu[d, nseg..E] = T
+ *      plan_expert       int32 [R, E]: expert of segment j, -1 past nseg
+ *      plan_wrow         int32 [R, E]: weight row of segment j, -1 past nseg
+ *                        (and -1 with EP_DEV_SLOTS if no slot was free)
+ *      plan_nseg         int32 [R]
+ *      slot_expert       int32 [R, B]: expert to prefetch into slot b, -1 if
+ *                        unused (may be NULL when B == 0)
+ *      status            EP_DEV_PLAN_TOTAL (slot_expert all -1, the other
+ *                        outputs left unwritten),
+ *                        EP_DEV_SLOTS
+ * One single-CTA kernel.
+ */
+EP_API int ep_plan_balanced(const int32_t* tokens_per_expert, int R, int S, int K,
+                     int E, int B, int32_t* plan_cu, int32_t* plan_expert,
+                     int32_t* plan_wrow, int32_t* plan_nseg,
+                     int32_t* slot_expert, int32_t* status, void* stream);
+
+/*
+ * ep_prefetch_weights -- fill the redundant-expert slots before the expert
+ * GEMMs ("MoonEP核心功能深度剖析", "快速上手": prefetch_weight(plan,
+ * full_gate_weight, full_up_weight, full_down_weight); "3. 智能内存管理",
+ * 图3: rows [E, E+B) are the local prefetch slots).
+ *
+ * in   slot_expert       int32 [R, B] from ep_plan_balanced
+ *      elems_per_expert  16-bit elements per expert row of one projection
+ *                        (H*I); elems_per_expert*2 % 16 == 0
+ * in/out gate, up, down  16-bit [E + R*B, elems_per_expert] each: row
+ *                        E + d*B + b <- row slot_expert[d,b] when that is
+ *                        >= 0; every other row is left as it is
+ *      num_sms           SMs to use, 0 = all
+ */
+EP_API int ep_prefetch_weights(const int32_t* slot_expert, int R, int E, int B,
+                        int64_t elems_per_expert, void* gate, void* up,
+                        void* down, int num_sms, void* stream);
+
+/* ---- diagnostics (used by the test-suite) ------------------------------ */
+
+/* out[i] = e4m3 code of x[i] through the same device conversion the FP8
+ * dispatch uses (round to nearest even, saturate to +-448). */
+EP_API int ep_debug_e4m3_encode(const float* x, uint8_t* out, int64_t n,
+                         void* stream);
+
+/* One thread polls *flag until it is non-zero, giving up after `max_polls`
+ * polls with EP_DEV_TIMEOUT OR-ed into *status: the bounded wait every
+ * device-side spin in this library uses, exposed so its give-up path can be
+ * exercised with a flag that nothing sets. */
+EP_API int ep_debug_bounded_wait(const int32_t* flag, int64_t max_polls,
+                          int32_t* status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EPLAYOUT_H_ */

@@ -1,0 +1,133 @@
+"""The C ABI library loads, exports every entry point its header declares,
+and rejects bad arguments on the host before touching the GPU. No compute
+call is made here: these tests run without a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import combine_ep_layout_09_b200 as ep
+from combine_ep_layout_09_b200 import build as epbuild
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include",
+                      "eplayout.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^EP_API [^;(]*?\b(ep_\w+)\s*\(", src,
+                                 flags=re.M)))
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for n in ["ep_layout", "ep_dispatch", "ep_combine", "ep_plan_balanced",
+              "ep_prefetch_weights", "ep_capacity_bound",
+              "ep_layout_workspace_bytes", "ep_strerror", "ep_abi_version"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(epbuild.LIB)
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_library_is_the_in_tree_build():
+    assert os.path.dirname(ep.library_path()) == os.path.dirname(
+        os.path.abspath(ep.__file__))
+    assert epbuild.up_to_date()
+
+
+def test_pure_host_entry_points():
+    assert ep.ep_abi_version() == 1
+    assert ep.ep_capacity_bound(32768, 8, 256, 128) == 32768 * 8 + 256 * 127
+    assert ep.ep_capacity_bound(10, 2, 4, 1) == 20
+    assert ep.ep_capacity_bound(-1, 2, 4, 1) < 0
+    assert ep.ep_layout_workspace_bytes(32768, 8, 256) > 0
+    assert ep.ep_layout_workspace_bytes(10, 0, 4) == 0
+    assert ep.ep_layout_workspace_bytes(10, 2, 4096) == 0   # E too large
+    for code in [0, -1, -2, -3, -4, -5, 1, 2, 4, 8, 16]:
+        assert ep.strerror(code) != "unknown code"
+
+
+def _raw():
+    return ctypes.CDLL(epbuild.LIB)
+
+
+def test_layout_rejects_on_host():
+    lib = _raw()
+    lib.ep_layout.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                              ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                              ctypes.c_void_p, ctypes.c_void_p,
+                              ctypes.c_void_p, ctypes.c_void_p,
+                              ctypes.c_int64, ctypes.c_void_p,
+                              ctypes.c_size_t, ctypes.c_void_p,
+                              ctypes.c_void_p]
+    fake = ctypes.c_void_p(1 << 20)        # aligned, never dereferenced
+    args = dict(R=4, S=8, K=2, E=8, pad=1, cap=64)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.ep_layout(fake, a["R"], a["S"], a["K"], a["E"], a["pad"],
+                             fake, fake, fake, fake, a["cap"], fake, 1 << 20,
+                             None, None)
+    assert call(E=10) == ep.EP_ERR_INVALID_ARG      # E % R != 0
+    assert call(K=0) == ep.EP_ERR_INVALID_ARG
+    assert call(K=33) == ep.EP_ERR_INVALID_ARG
+    assert call(pad=0) == ep.EP_ERR_INVALID_ARG
+    assert call(cap=63) == ep.EP_ERR_CAPACITY       # below N*K
+    assert call(pad=4, cap=64) == ep.EP_ERR_CAPACITY
+    assert call(cap=2 ** 31) == ep.EP_ERR_CAPACITY
+    assert call(S=1 << 28, cap=1 << 31) == ep.EP_ERR_INVALID_ARG
+
+
+def test_dispatch_combine_reject_on_host():
+    lib = _raw()
+    P, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    lib.ep_dispatch.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i32,
+                                P, P, P, i32, P, P]
+    lib.ep_combine.argtypes = [P, P, P, i64, i32, i32, i64, P, i32, P, P]
+    ok = ctypes.c_void_p(1 << 20)
+    bad = ctypes.c_void_p((1 << 20) + 8)
+    # fp8 needs H % 128 == 0
+    assert lib.ep_dispatch(ok, ok, ok, ok, ok, 4, 2, 8, 200, 16, 1, ok, ok,
+                           ok, 0, None, None) == ep.EP_ERR_INVALID_ARG
+    # misaligned receive buffer
+    assert lib.ep_dispatch(ok, ok, ok, ok, ok, 4, 2, 8, 256, 16, 0, bad, None,
+                           None, 0, None, None) == ep.EP_ERR_ALIGNMENT
+    # fp8 without scales
+    assert lib.ep_dispatch(ok, ok, ok, ok, ok, 4, 2, 8, 256, 16, 1, ok, None,
+                           None, 0, None, None) == ep.EP_ERR_ALIGNMENT
+    assert lib.ep_combine(ok, ok, ok, 4, 2, 12, 16, ok, 0, None,
+                          None) == ep.EP_ERR_INVALID_ARG   # H % 8
+    assert lib.ep_combine(ok, ok, ok, 4, 2, 16, 16, bad, 0, None,
+                          None) == ep.EP_ERR_ALIGNMENT
+    assert lib.ep_combine(ok, ok, ok, 0, 2, 16, 16, ok, 0, None,
+                          None) == ep.EP_OK                # nothing to do
+
+
+def test_plan_prefetch_reject_on_host():
+    lib = _raw()
+    P, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    lib.ep_plan_balanced.argtypes = [P, i32, i32, i32, i32, i32, P, P, P, P,
+                                     P, P, P]
+    lib.ep_prefetch_weights.argtypes = [P, i32, i32, i32, i64, P, P, P, i32, P]
+    ok = ctypes.c_void_p(1 << 20)
+    assert lib.ep_plan_balanced(ok, 0, 4, 2, 8, 1, ok, ok, ok, ok, ok, None,
+                                None) == ep.EP_ERR_INVALID_ARG
+    assert lib.ep_plan_balanced(ok, 2, 4, 2, 8, 1, ok, ok, ok, ok, None, None,
+                                None) == ep.EP_ERR_ALIGNMENT
+    assert lib.ep_prefetch_weights(ok, 2, 8, 1, 7, ok, ok, ok, 0,
+                                   None) == ep.EP_ERR_INVALID_ARG
+    assert lib.ep_prefetch_weights(ok, 2, 8, 0, 8, ok, ok, ok, 0,
+                                   None) == ep.EP_OK
+
+
+def test_binding_rejects_host_tensors():
+    import torch
+    t = torch.zeros(8, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        ep.ep_layout(t, 1, 4, 2, 2, 1, t, t, t, t, torch.zeros(
+            64, dtype=torch.uint8))

@@ -1,0 +1,97 @@
+"""GPU combine against the oracle: the same fp32 fused-multiply-add chain in
+k order, so results are bit-identical; the stated bar (within 1 bf16 ulp of
+the exact sum, absolute error <= 1e-2 * max|y|) is checked as well."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from gpu_util import (DEV, gpu_combine, gpu_layout, rows_to_host, to_bf16_dev,
+                      to_dev, u16)
+
+pytestmark = pytest.mark.gpu
+
+
+def as_f32(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+def ulp_bf16(v):
+    a = np.abs(v)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.exp2(np.maximum(e, -126) - 7)
+
+
+def check(y_bits, pos, w, num_sms=0):
+    N, K = pos.shape
+    out, st = gpu_combine(to_bf16_dev(y_bits), to_dev(pos), to_dev(w), N, K,
+                          num_sms=num_sms)
+    assert st == 0
+    got = u16(out)
+    ref = oracle.combine(y_bits, pos, w)
+    np.testing.assert_array_equal(got, ref)          # bit-exact
+    # the stated tolerance against the exact (double) sum
+    exact = oracle.combine_f64(y_bits, pos, w)
+    err = np.abs(as_f32(got).astype(np.float64) - exact)
+    maxabs = float(np.abs(as_f32(y_bits)).max()) if y_bits.size else 0.0
+    assert np.all(err <= 1e-2 * maxabs + 1e-30)
+    return got
+
+
+@pytest.mark.parametrize("N,K,H,rows", [
+    (1, 1, 8, 1), (256, 2, 256, 600), (1000, 8, 7168, 9000),
+    (333, 3, 520, 1200), (77, 5, 24, 400), (129, 9, 1024, 2000),
+    (64, 32, 64, 3000), (500, 6, 4096, 3100), (40, 4, 16, 100),
+])
+def test_random(N, K, H, rows):
+    rng = np.random.default_rng(N + K + H)
+    y = u16(workloads.bf16_normal((rows, H), N + H))
+    pos = rng.integers(0, rows, size=(N, K)).astype(np.int32)
+    w = rng.random((N, K)).astype(np.float32)
+    check(y, pos, w)
+
+
+def test_skipped_entries_and_limited_sms():
+    rng = np.random.default_rng(2)
+    y = u16(workloads.bf16_normal((300, 512), 3))
+    pos = rng.integers(0, 300, size=(200, 8)).astype(np.int32)
+    pos[rng.random(pos.shape) < 0.2] = -1
+    pos[5] = -1                                   # a token with no entries
+    w = (rng.standard_normal((200, 8))).astype(np.float32)
+    got = check(y, pos, w, num_sms=2)
+    assert np.all(got[5] == 0)
+
+
+def test_k_order_and_fma_cases():
+    # 1 - 1 + 2^-30 (order) and the 31-bit product case (fusion)
+    y = np.array([[0x3F80] * 8, [0xBF80] * 8, [0x3080] * 8, [0x3F81] * 8],
+                 np.uint16)
+    pos = np.array([[0, 1, 2], [2, 1, 0]], np.int32)
+    w = np.ones((2, 3), np.float32)
+    got = check(y, pos, w)
+    assert as_f32(got)[0, 0] == 2.0 ** -30 and as_f32(got)[1, 0] == 0.0
+    pos = np.array([[3, 3]], np.int32)
+    w = np.array([[-(1 + 2.0 ** -23), 1 + 2.0 ** -23]], np.float32)
+    got = check(y, pos, w)
+    assert as_f32(got)[0, 0] == 2.0 ** -30
+
+
+@pytest.mark.parametrize("name", ["prefill", "decode"])
+def test_full_size_sampled(name):
+    wl = workloads.WORKLOADS[name]
+    topk, w = workloads.routing(wl)
+    g = gpu_layout(topk, wl.R, wl.S, wl.E, 1)
+    cap = g["dev"]["cap"]
+    y = workloads.expert_outputs(cap, wl.H, wl.seed, device="cuda:0")
+    out, st = gpu_combine(y, g["dev"]["pos"], to_dev(w), wl.N, wl.K)
+    assert st == 0
+    o_lay = oracle.layout(topk, wl.E, 1, cap)
+    rng = np.random.default_rng(1)
+    toks = np.sort(rng.choice(wl.N, min(wl.N, 512), replace=False))
+    toks[0], toks[-1] = 0, wl.N - 1
+    rows = o_lay["pos"][toks].ravel()
+    ysel = rows_to_host(y, rows)
+    pos_small = np.arange(len(rows), dtype=np.int32).reshape(len(toks), wl.K)
+    ref = oracle.combine(ysel, pos_small, w[toks])
+    np.testing.assert_array_equal(rows_to_host(out, toks), ref)

@@ -1,0 +1,144 @@
+"""GPU dispatch (bf16 copy and fused FP8 quantisation) against the oracle:
+bit-exact payload, scales and weights; padding rows zero; rows past the used
+region untouched."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from gpu_util import (RECV_BF16_FILL, RECV_FP8_FILL, RECV_W_FILL, SCALE_FILL,
+                      gpu_dispatch, gpu_layout, rows_to_host, to_bf16_dev, u16)
+
+pytestmark = pytest.mark.gpu
+
+
+def make(seed, R, S, K, E, H, scale=1.0, distinct=False):
+    rng = np.random.default_rng(seed)
+    topk, w = workloads.random_topk(rng, R * S, K, E, distinct=distinct)
+    hid = workloads.bf16_normal((R * S, H), seed) * scale
+    return topk, w, u16(hid.to(torch.bfloat16))
+
+
+def check_full(topk, w, hidden, R, S, E, H, pad, fp8, num_sms=0,
+               with_weights=True):
+    N, K = topk.shape
+    g = gpu_layout(topk, R, S, E, pad)
+    cap = g["dev"]["cap"]
+    d = gpu_dispatch(to_bf16_dev(hidden), w, g, E, fp8,
+                     with_weights=with_weights, num_sms=num_sms)
+    assert d["status"] == 0
+    o_lay = oracle.layout(topk, E, pad, cap)
+    if fp8:
+        r, s, rw = oracle.dispatch_fp8(hidden, w, o_lay, E, cap,
+                                       recv_fill=RECV_FP8_FILL,
+                                       scale_fill=SCALE_FILL,
+                                       recv_w_fill=RECV_W_FILL)
+        np.testing.assert_array_equal(d["recv"].cpu().numpy()[:cap], r)
+        np.testing.assert_array_equal(d["scales"].cpu().numpy()[:cap], s)
+    else:
+        r, rw = oracle.dispatch_bf16(hidden, w, o_lay, E, cap,
+                                     recv_fill=RECV_BF16_FILL,
+                                     recv_w_fill=RECV_W_FILL)
+        np.testing.assert_array_equal(u16(d["recv"])[:cap], r)
+    if with_weights:
+        np.testing.assert_array_equal(d["recv_w"].cpu().numpy()[:cap], rw)
+
+
+@pytest.mark.parametrize("R,S,K,E,H,pad", [
+    (4, 64, 2, 8, 256, 1),          # tiny shape
+    (2, 700, 8, 16, 7168, 1),       # several tiles, full row width
+    (3, 333, 5, 9, 520, 3),         # row not a multiple of 512 channels
+    (2, 257, 3, 8, 8, 4),           # one 16-byte vector per row
+    (4, 100, 4, 16, 24, 128),       # odd vector count, heavy padding
+    (1, 1, 1, 1, 16, 1),
+])
+def test_bf16(R, S, K, E, H, pad):
+    topk, w, h = make(R + S + K + E + H, R, S, K, E, H)
+    check_full(topk, w, h, R, S, E, H, pad, fp8=False)
+
+
+@pytest.mark.parametrize("R,S,K,E,H,pad", [
+    (4, 64, 2, 8, 256, 1),
+    (2, 700, 8, 16, 7168, 1),
+    (3, 333, 5, 9, 384, 3),
+    (2, 301, 8, 32, 640, 128),
+    (1, 1, 1, 1, 128, 1),
+])
+def test_fp8(R, S, K, E, H, pad):
+    topk, w, h = make(7 * (R + S + K + E + H), R, S, K, E, H)
+    check_full(topk, w, h, R, S, E, H, pad, fp8=True)
+
+
+def test_fp8_extreme_values():
+    # huge, tiny, subnormal and zero groups, signed zeros, exact ties
+    R, S, K, E, H = 2, 40, 3, 4, 512
+    rng = np.random.default_rng(3)
+    topk, w = workloads.random_topk(rng, R * S, K, E)
+    x = rng.standard_normal((R * S, H)).astype(np.float32)
+    x[0] *= 1e30
+    x[1] *= 1e-30
+    x[2, :128] = 0.0
+    x[2, 128:256] = -0.0
+    x[3] = 0.0
+    x[4, 0] = 1.0
+    x[4, 1:128] = 1.0 / 448 * 1.0625       # exact ties after scaling
+    x[5, :] = 3e-39                        # bf16 subnormal group
+    x[6, ::2] = -x[6, ::2]
+    h = (x.view(np.uint32) >> 16).astype(np.uint16)   # truncate to bf16
+    check_full(topk, w, h, R, S, E, H, 1, fp8=True)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_without_weights_and_limited_sms(fp8):
+    topk, w, h = make(99, 2, 500, 4, 8, 1024)
+    check_full(topk, w, h, 2, 500, 8, 1024, 16, fp8=fp8, num_sms=3,
+               with_weights=False)
+
+
+def test_decode_full_size():
+    wl = workloads.WORKLOADS["decode"]
+    topk, w = workloads.routing(wl)
+    h = u16(workloads.hidden_states(wl))
+    check_full(topk, w, h, wl.R, wl.S, wl.E, wl.H, wl.pad, fp8=True)
+
+
+@pytest.mark.parametrize("name", ["prefill", "skewed"])
+def test_full_size_sampled(name):
+    wl = workloads.WORKLOADS[name]
+    topk, w = workloads.routing(wl)
+    hid_dev = workloads.hidden_states(wl, device="cuda:0")
+    g = gpu_layout(topk, wl.R, wl.S, wl.E, wl.pad)
+    cap = g["dev"]["cap"]
+    d = gpu_dispatch(hid_dev, w, g, wl.E, wl.fp8)
+    assert d["status"] == 0
+    o_lay = oracle.layout(topk, wl.E, wl.pad, cap)
+    used = int(o_lay["offsets"][-1])
+    # all weights, every row: recv_w[pos[t,k]] == w[t,k], padding 0, tail
+    rw = d["recv_w"].cpu().numpy()
+    np.testing.assert_array_equal(rw[o_lay["pos"]], w)
+    assert np.all(rw[:used][o_lay["row_src"][:used] < 0] == 0)
+    assert np.all(rw[used:] == RECV_W_FILL)
+    # sampled tokens: the K destination rows against the oracle
+    rng = np.random.default_rng(0)
+    toks = np.sort(rng.choice(wl.N, 384, replace=False))
+    toks[0], toks[-1] = 0, wl.N - 1
+    hrows = u16(hid_dev.index_select(0, torch.from_numpy(toks).cuda()))
+    rows = o_lay["pos"][toks].ravel()
+    if wl.fp8:
+        q, s = oracle.quantize_rows(hrows)
+        np.testing.assert_array_equal(rows_to_host(d["recv"], rows),
+                                      np.repeat(q, wl.K, axis=0))
+        np.testing.assert_array_equal(rows_to_host(d["scales"], rows),
+                                      np.repeat(s, wl.K, axis=0))
+        # every used row was written: scales are >= 0, not the fill
+        sc = d["scales"][:used]
+        assert bool((sc >= 0).all())
+        assert bool((d["scales"][used:] == SCALE_FILL).all())
+    else:
+        np.testing.assert_array_equal(rows_to_host(d["recv"], rows),
+                                      np.repeat(hrows, wl.K, axis=0))
+        pad_rows = np.where(o_lay["row_src"][:used] < 0)[0]
+        assert len(pad_rows) > 0
+        sel = rows_to_host(d["recv"], pad_rows[:2000])
+        assert np.all(sel == 0)
