@@ -569,10 +569,14 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-tokens", type=int, default=8192)
+    ap.add_argument("--tokens-per-rank", type=int, default=None,
+                    help="override S (smaller cases for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     wl = workloads.WORKLOADS[args.workload]
+    if args.tokens_per_rank:
+        wl = workloads.scaled(wl, S=args.tokens_per_rank)
 
     if args.impl == "reference":
         res = run_reference(args, wl)
