@@ -111,6 +111,37 @@ EP_API int ep_layout(const int32_t* topk_experts, int R, int S, int K, int E,
               int32_t* status, void* stream);
 
 /*
+ * ep_layout_static -- ep_layout for callers that cannot allocate device
+ * memory. The pages have no counterpart to this entry point; it exists for
+ * users of this library whose code may not call cudaMalloc: a plugin inside
+ * a host framework that owns all device memory, a serving runtime that plans
+ * every byte up front and forbids allocation on its request path, or code
+ * running while a CUDA graph is captured in global mode.
+ *
+ * Same arguments, results and errors as ep_layout, minus the workspace: the
+ * scratch is a fixed array inside the library's device image, of
+ * EP_LAYOUT_STATIC_SCRATCH_BYTES per GPU, held from the library's first use
+ * on a GPU until the process exits. Nothing is allocated by the call.
+ *   - Limit: problems with ep_layout_workspace_bytes(R*S, K, E) larger than
+ *     EP_LAYOUT_STATIC_SCRATCH_BYTES are refused with EP_ERR_WORKSPACE
+ *     before any CUDA call (E=256 fits up to about 4.2 M entries N*K).
+ *   - The first call on each GPU looks up the array's device address
+ *     (cudaGetSymbolAddress, with that GPU current) and caches it; make that
+ *     first call before any stream capture.
+ *   - All calls on a GPU share the array and it keeps the last call's
+ *     contents. Each call clears what must start at zero, but two calls that
+ *     overlap on the GPU (different streams, unordered host threads) race
+ *     and corrupt each other: order them on one stream.
+ */
+#define EP_LAYOUT_STATIC_SCRATCH_BYTES (1u << 20)
+EP_API int ep_layout_static(const int32_t* topk_experts, int R, int S, int K,
+                            int E, int token_padding,
+                            int32_t* tokens_per_expert,
+                            int32_t* expert_offsets, int32_t* pos,
+                            int32_t* row_src, int64_t cap, int32_t* status,
+                            void* stream);
+
+/*
  * ep_dispatch -- step 4: copy every token row to its K receive rows
  * ("Экспертный параллелизм (EP)", "Что подтверждено": token activations are
  * sent to the experts; "DeepSeek开源周第二天：DeepEP深度分析", "性能": FP8
