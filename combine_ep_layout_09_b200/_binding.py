@@ -90,6 +90,8 @@ def _declare(L):
     L.ep_prefetch_weights.argtypes = [P, i32, i32, i32, i64, P, P, P, i32, P]
     L.ep_debug_e4m3_encode.restype = i32
     L.ep_debug_e4m3_encode.argtypes = [P, P, i64, P]
+    L.ep_debug_quantize.restype = i32
+    L.ep_debug_quantize.argtypes = [P, P, P, i64, P]
     L.ep_debug_bounded_wait.restype = i32
     L.ep_debug_bounded_wait.argtypes = [P, i64, P, P]
 
@@ -260,6 +262,14 @@ def ep_debug_e4m3_encode(x, out, stream=None):
         _ptr(x, "x", _F32), _ptr(out, "out", (torch.uint8,), x.numel()),
         x.numel(), _stream(stream))
     _check(rc, "ep_debug_e4m3_encode")
+
+
+def ep_debug_quantize(x, group_scale, out, stream=None):
+    n = x.numel()
+    rc = lib().ep_debug_quantize(
+        _ptr(x, "x", _F32), _ptr(group_scale, "group_scale", _F32, n // 16),
+        _ptr(out, "out", (torch.uint8,), n), n, _stream(stream))
+    _check(rc, "ep_debug_quantize")
 
 
 def ep_debug_bounded_wait(flag, max_polls, status, stream=None):

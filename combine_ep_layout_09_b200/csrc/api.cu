@@ -191,6 +191,16 @@ int ep_debug_e4m3_encode(const float* x, uint8_t* out, int64_t n,
   return cuda_rc(ep::launch_debug_e4m3(x, out, n, as_stream(stream)));
 }
 
+int ep_debug_quantize(const float* x, const float* group_scale, uint8_t* out,
+                      int64_t n, void* stream) {
+  if (n < 0 || n % 16 != 0) return EP_ERR_INVALID_ARG;
+  if (n == 0) return EP_OK;
+  if (!aligned16(x) || !aligned16(group_scale) || !aligned16(out))
+    return EP_ERR_ALIGNMENT;
+  return cuda_rc(ep::launch_debug_quantize(x, group_scale, out, n,
+                                           as_stream(stream)));
+}
+
 int ep_debug_bounded_wait(const int32_t* flag, int64_t max_polls,
                           int32_t* status, void* stream) {
   if (max_polls < 0) return EP_ERR_INVALID_ARG;

@@ -3,17 +3,37 @@
 //
 // "Экспертный параллелизм (EP)", section "Что подтверждено": activations,
 // not expert weights, travel to the experts. "DeepSeek开源周第二天：DeepEP深度
-// 分析", section "性能": FP8 dispatch. "MoonEP核心功能深度剖析", section
-// "2. 高效通信机制": rows land directly in their final expert-grouped
-// position (computed by the layout kernels), no later permutation.
+// 分析", section "性能": FP8 dispatch; section "代码解读": data movement through
+// the TMA engine. "MoonEP核心功能深度剖析", section "2. 高效通信机制": rows land
+// directly in their final expert-grouped position (computed by the layout
+// kernels), with no later permutation.
 //
-// One persistent CTA per (SM, slot). Its producer lane streams whole token
-// rows global -> shared with 1-D bulk copies (TMA engine) into a ring of
-// mbarrier-tracked stages; the consumer warps read a row from shared memory
-// once, quantise it in registers when FP8 is asked for, and write each of its
-// K destination rows with 16-byte stores. Reads are 1/(K+1) of the bytes, so
-// the kernel is bound by HBM write bandwidth. Padding rows are zero-filled at
-// the end by all warps.
+// Both kernels move rows with the TMA engine's 1-D bulk copies (no tensor
+// map, no multicast): a token row comes into shared memory once and leaves
+// K times. The kernel reads 1/(K+1) of the bytes it moves, so HBM write
+// bandwidth bounds it.
+//
+//   k_dispatch_bf16  one-warp CTAs; lane 0 keeps a ring of token rows in
+//                    flight and, per row, issues K bulk stores from shared
+//                    memory to the destination rows. No data passes through
+//                    registers.
+//   k_dispatch_fp8   a producer warp streams rows in; consumer warps
+//                    quantise their 512-channel slice into an output stage
+//                    in shared memory (codes, then the row's scales); one
+//                    thread bulk-stores that stage K times.
+//
+// Quantisation ("bracketed reciprocal"): the code must be e4m3(RN(x/s)) with
+// the fp32 quotient correctly rounded. With inv = RN(1/s), the products
+// lo = RN(x * RN(inv*(1-2^-20))) and hi = RN(x * RN(inv*(1+2^-20))) enclose
+// RN(x/s) (each rounding moves a value by at most 2^-24 relative, far
+// inside the 2^-20 margin). Rounding to E4M3 is monotone, so when lo and hi
+// encode to the same code that code is e4m3(RN(x/s)). Otherwise the pair is
+// recomputed with the correctly rounded division __fdiv_rn. That happens
+// for about 3e-5 of the values, the ones within 2^-20 of a rounding
+// boundary. Values in the fp32 subnormal range all encode to +-0 on the
+// correct side, so the bracket needs no normal-range assumption there. A
+// scale below 2^-125, whose reciprocal could overflow, takes the division
+// path for the whole group.
 #include <algorithm>
 
 #include "ep_device.cuh"
@@ -22,165 +42,100 @@
 namespace ep {
 namespace {
 
-constexpr int kUnitCh = 512;            // channels one warp covers per pass
-constexpr int kMaxConsumerWarps = 16;   // H/512 rounded up, capped
+constexpr int kUnitCh = 512;           // channels one warp covers per pass
+constexpr int kMaxConsumerWarps = 16;  // H/512 rounded up, capped
 constexpr int kMaxStages = 8;
-constexpr size_t kStageBudget = 100 * 1024;  // shared bytes for the ring
 
 __host__ __device__ constexpr uint32_t align128(uint32_t x) {
   return (x + 127u) & ~127u;
 }
 
-// Quantise 16 channels held by this lane; lanes 8g..8g+7 of the warp hold the
-// 128 channels of one group. Returns the 16 codes, writes the group scale.
-__device__ __forceinline__ uint4 quantize16(const uint4& a, const uint4& b,
-                                            float& scale_out) {
-  float x[16];
+__device__ __forceinline__ void named_barrier(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// E4M3 quantisation of 16 values by one group scale (shared with the
+// diagnostic entry point so that the tests exercise this exact code)
+// ---------------------------------------------------------------------------
+
+struct GroupScale {
+  float scale;   // the group's fp32 scale
+  float inv_lo;  // RN(RN(1/scale) * (1 - 2^-20))
+  float inv_hi;  // RN(RN(1/scale) * (1 + 2^-20))
+  bool bracket;  // reciprocal path valid (scale >= 2^-125)
+};
+
+__device__ __forceinline__ GroupScale make_group_scale(float scale) {
+  GroupScale g;
+  g.scale = scale;
+  g.bracket = scale >= 0x1p-125f;
+  const float inv = g.bracket ? __frcp_rn(scale) : 0.0f;
+  g.inv_lo = inv * (1.0f - 0x1p-20f);
+  g.inv_hi = inv * (1.0f + 0x1p-20f);
+  return g;
+}
+
+// Two codes (low byte = a) for e4m3(RN(a/scale)), e4m3(RN(b/scale)).
+__device__ __forceinline__ uint32_t codes2_exact(float a, float b,
+                                                 const GroupScale& g) {
+  return e4m3x2(__fdiv_rn(a, g.scale), __fdiv_rn(b, g.scale));
+}
+
+// 16 codes of x[0..15] (scale != 0); bytes in channel order.
+__device__ __forceinline__ uint4 quantize16(const float (&x)[16],
+                                            const GroupScale& g) {
+  uint32_t c[8];
+  bool agree = g.bracket;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t lo = e4m3x2(x[2 * i] * g.inv_lo, x[2 * i + 1] * g.inv_lo);
+    const uint32_t hi = e4m3x2(x[2 * i] * g.inv_hi, x[2 * i + 1] * g.inv_hi);
+    agree = agree && (lo == hi);
+    c[i] = lo;
+  }
+  if (!agree) {  // rare: some value sits on a rounding boundary
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t lo = e4m3x2(x[2 * i] * g.inv_lo, x[2 * i + 1] * g.inv_lo);
+      const uint32_t hi = e4m3x2(x[2 * i] * g.inv_hi, x[2 * i + 1] * g.inv_hi);
+      if (!g.bracket || lo != hi) c[i] = codes2_exact(x[2 * i], x[2 * i + 1], g);
+    }
+  }
+  return make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16),
+                    c[4] | (c[5] << 16), c[6] | (c[7] << 16));
+}
+
+// Unpack 16 bf16 (two 16-byte words) to fp32; returns max |x|.
+__device__ __forceinline__ float unpack16(const uint4& a, const uint4& b,
+                                          float (&x)[16]) {
   const uint32_t wd[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     x[2 * i] = bf16_lo(wd[i]);
     x[2 * i + 1] = bf16_hi(wd[i]);
+    amax = fmaxf(amax, fmaxf(fabsf(x[2 * i]), fabsf(x[2 * i + 1])));
   }
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-  const float scale = __fdiv_rn(amax, 448.0f);
-  scale_out = scale;
-  uint4 q = make_uint4(0u, 0u, 0u, 0u);
-  if (scale != 0.0f) {
-    uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t lo = e4m3x2(__fdiv_rn(x[4 * i], scale),
-                                 __fdiv_rn(x[4 * i + 1], scale));
-      const uint32_t hi = e4m3x2(__fdiv_rn(x[4 * i + 2], scale),
-                                 __fdiv_rn(x[4 * i + 3], scale));
-      w[i] = lo | (hi << 16);
-    }
-    q = make_uint4(w[0], w[1], w[2], w[3]);
-  }
-  return q;
+  return amax;
 }
 
+// ---------------------------------------------------------------------------
+// padding rows: zero payload, zero scales, zero weight (all warps of the grid)
+// ---------------------------------------------------------------------------
+
 template <bool kFp8>
-__global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32)
-    k_dispatch(const uint16_t* __restrict__ hidden, const float* __restrict__ w,
-               const int32_t* __restrict__ pos, const int32_t* __restrict__ row_src,
-               const int32_t* __restrict__ offsets, int64_t N, int K, int E,
-               int H, int64_t cap, uint8_t* __restrict__ recv,
-               float* __restrict__ scales, float* __restrict__ recv_w,
-               int stages, int32_t* __restrict__ status) {
-  extern __shared__ __align__(128) uint8_t smem[];
+__device__ void zero_padding_rows(const int32_t* __restrict__ row_src,
+                                  const int32_t* __restrict__ offsets, int E,
+                                  int H, int64_t cap, uint8_t* __restrict__ recv,
+                                  float* __restrict__ scales,
+                                  float* __restrict__ recv_w) {
+  const int lane = threadIdx.x & 31;
   const int nwarps = blockDim.x >> 5;
-  const int cw = nwarps - 1;  // consumer warps; the last warp produces
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t row_bytes = uint32_t(H) * 2u;
-  const uint32_t stage_bytes = align128(row_bytes);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(stages) * stage_bytes);
-  uint64_t* empty = full + kMaxStages;
-  const int G = H >> 7;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < stages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], uint32_t(cw));
-    }
-    fence_mbar_init();
-  }
-  __syncthreads();
-
-  if (warp == cw) {
-    // ---- producer: one lane keeps `stages` token rows in flight ----------
-    if (lane == 0) {
-      int it = 0;
-      bool ok = true;
-      for (int64_t t = blockIdx.x; t < N; t += gridDim.x, ++it) {
-        const int s = it % stages;
-        const uint32_t ph = uint32_t(it / stages) & 1u;
-        if (it >= stages && !mbar_wait_bounded(&empty[s], ph ^ 1u)) {
-          report(status, EP_DEV_TIMEOUT);
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(&full[s], row_bytes);
-        bulk_g2s(smem + size_t(s) * stage_bytes, hidden + t * H, row_bytes, &full[s]);
-      }
-      // Drain: never leave the CTA with a bulk copy still writing its smem.
-      if (!ok || true) {
-        const int issued = it;
-        for (int s = 0; s < stages && s < issued; ++s) {
-          const int last = issued - 1 - ((issued - 1 - s) % stages);
-          if (!mbar_wait_bounded(&full[s], uint32_t(last / stages) & 1u))
-            report(status, EP_DEV_TIMEOUT);
-        }
-      }
-    }
-    __syncwarp();
-  } else {
-    // ---- consumers -----------------------------------------------------
-    int it = 0;
-    for (int64_t t = blockIdx.x; t < N; t += gridDim.x, ++it) {
-      const int s = it % stages;
-      const uint32_t ph = uint32_t(it / stages) & 1u;
-      int p_l = -1;
-      float w_l = 0.0f;
-      if (lane < K) {
-        p_l = __ldg(pos + t * K + lane);
-        w_l = __ldg(w + t * K + lane);
-        if (p_l >= cap) {
-          report(status, EP_DEV_CAPACITY);
-          p_l = -1;
-        }
-      }
-      if (!mbar_wait_bounded(&full[s], ph)) {
-        report(status, EP_DEV_TIMEOUT);
-        break;
-      }
-      const uint8_t* row = smem + size_t(s) * stage_bytes;
-      for (int u = warp; u * kUnitCh < H; u += cw) {
-        const int c0 = u * kUnitCh + lane * 16;  // first channel of this lane
-        const bool act0 = c0 < H;
-        const bool act1 = c0 + 8 < H;
-        uint4 a = make_uint4(0u, 0u, 0u, 0u), b = a;
-        if (act0) a = *reinterpret_cast<const uint4*>(row + size_t(c0) * 2);
-        if (act1) b = *reinterpret_cast<const uint4*>(row + size_t(c0) * 2 + 16);
-        if constexpr (kFp8) {
-          float scale;
-          const uint4 q = quantize16(a, b, scale);  // whole warp (shuffles)
-          const int g = c0 >> 7;
-          for (int k = 0; k < K; ++k) {
-            const int p = __shfl_sync(0xffffffffu, p_l, k);
-            if (p < 0) continue;
-            if (act0) {
-              st_v4(recv + int64_t(p) * H + c0, q);
-              if ((lane & 7) == 0) scales[int64_t(p) * G + g] = scale;
-            }
-          }
-        } else {
-          uint16_t* recv16 = reinterpret_cast<uint16_t*>(recv);
-          for (int k = 0; k < K; ++k) {
-            const int p = __shfl_sync(0xffffffffu, p_l, k);
-            if (p < 0) continue;
-            uint16_t* dst = recv16 + int64_t(p) * H + c0;
-            if (act0) st_v4(dst, a);
-            if (act1) st_v4(dst + 8, b);
-          }
-        }
-      }
-      if (warp == 0 && lane < K && p_l >= 0 && recv_w) recv_w[p_l] = w_l;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-    }
-  }
-
-  // ---- padding rows (row_src == -1 below off[E]): zeros ------------------
   const int64_t used = min(int64_t(__ldg(offsets + E)), cap);
-  const int64_t gw = int64_t(blockIdx.x) * nwarps + warp;
+  const int64_t gw = int64_t(blockIdx.x) * nwarps + (threadIdx.x >> 5);
   const int64_t gstride = int64_t(gridDim.x) * nwarps;
+  const int G = H >> 7;
   const uint4 z = make_uint4(0u, 0u, 0u, 0u);
   for (int64_t r0 = gw * 32; r0 < used; r0 += gstride * 32) {
     const int64_t r = r0 + lane;
@@ -202,20 +157,289 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32)
   }
 }
 
-struct DispatchCfg {
+// ---------------------------------------------------------------------------
+// bf16: a pure TMA copy, one warp per CTA
+// ---------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(32)
+    k_dispatch_bf16(const uint16_t* __restrict__ hidden,
+                    const float* __restrict__ w, const int32_t* __restrict__ pos,
+                    const int32_t* __restrict__ row_src,
+                    const int32_t* __restrict__ offsets, int64_t N, int K,
+                    int E, int H, int64_t cap, uint8_t* __restrict__ recv,
+                    float* __restrict__ recv_w, int stages,
+                    int32_t* __restrict__ status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int lane = threadIdx.x;
+  const uint32_t row_bytes = uint32_t(H) * 2u;
+  const uint32_t stage_bytes = align128(row_bytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(stages) * stage_bytes);
+  const int64_t first = blockIdx.x, stride = gridDim.x;
+  const int64_t n_mine = first < N ? (N - 1 - first) / stride + 1 : 0;
+
+  if (lane == 0) {
+    for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
+    fence_mbar_init();
+    for (int64_t i = 0; i < stages && i < n_mine; ++i) {
+      mbar_arrive_expect_tx(&full[i], row_bytes);
+      bulk_g2s(smem + size_t(i) * stage_bytes, hidden + (first + i * stride) * H,
+               row_bytes, &full[i]);
+    }
+  }
+  __syncwarp();
+
+  bool ok = true;
+  for (int64_t i = 0; i < n_mine && ok; ++i) {
+    const int64_t t = first + i * stride;
+    const int s = int(i % stages);
+    int p_l = -1;
+    float w_l = 0.0f;
+    if (lane < K) {
+      p_l = __ldg(pos + t * K + lane);
+      w_l = __ldg(w + t * K + lane);
+      if (p_l >= cap) {
+        report(status, EP_DEV_CAPACITY);
+        p_l = -1;
+      }
+    }
+    if (lane == 0) ok = mbar_wait_bounded(&full[s], uint32_t(i / stages) & 1u);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) {
+      if (lane == 0) report(status, EP_DEV_TIMEOUT);
+      break;
+    }
+    for (int k = 0; k < K; ++k) {
+      const int p = __shfl_sync(0xffffffffu, p_l, k);
+      if (lane == 0 && p >= 0)
+        bulk_s2g(recv + int64_t(p) * row_bytes, smem + size_t(s) * stage_bytes,
+                 row_bytes);
+    }
+    if (lane == 0) {
+      bulk_commit();
+      // Refill the stage of the previous row once its stores have read it.
+      const int64_t nxt = i - 1 + stages;
+      if (i >= 1 && nxt < n_mine) {
+        const int sp = int((i - 1) % stages);
+        bulk_wait_read<1>();
+        mbar_arrive_expect_tx(&full[sp], row_bytes);
+        bulk_g2s(smem + size_t(sp) * stage_bytes, hidden + (first + nxt * stride) * H,
+                 row_bytes, &full[sp]);
+      }
+    }
+    if (lane < K && p_l >= 0 && recv_w) recv_w[p_l] = w_l;
+  }
+  if (lane == 0) {
+    // Loads still in flight after a give-up, then all stores complete.
+    if (!ok) {
+      for (int64_t i = 0; i < stages && i < n_mine; ++i) {
+        const int64_t last = n_mine - 1 - ((n_mine - 1 - i) % stages);
+        mbar_wait_bounded(&full[i], uint32_t(last / stages) & 1u);
+      }
+    }
+    bulk_wait_all<0>();
+  }
+  __syncwarp();
+  zero_padding_rows<false>(row_src, offsets, E, H, cap, recv, nullptr, recv_w);
+}
+
+// ---------------------------------------------------------------------------
+// fp8: producer warp + consumer warps, output stage bulk-stored K times
+// ---------------------------------------------------------------------------
+
+__global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32)
+    k_dispatch_fp8(const uint16_t* __restrict__ hidden,
+                   const float* __restrict__ w, const int32_t* __restrict__ pos,
+                   const int32_t* __restrict__ row_src,
+                   const int32_t* __restrict__ offsets, int64_t N, int K, int E,
+                   int H, int64_t cap, uint8_t* __restrict__ recv,
+                   float* __restrict__ scales, float* __restrict__ recv_w,
+                   int s_in, int s_out, int32_t* __restrict__ status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int nwarps = blockDim.x >> 5;
+  const int cw = nwarps - 1;  // consumer warps; the last warp produces
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = H >> 7;
+  const uint32_t row_bytes = uint32_t(H) * 2u;
+  const uint32_t in_bytes = align128(row_bytes);
+  const uint32_t scale_bytes = uint32_t(G) * 4u;
+  const uint32_t out_bytes = align128(uint32_t(H) + scale_bytes);
+  uint8_t* in_base = smem;
+  uint8_t* out_base = smem + size_t(s_in) * in_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(out_base + size_t(s_out) * out_bytes);
+  uint64_t* empty = full + kMaxStages;
+  // Bulk stores need 16-byte multiples; the scales of a row qualify when
+  // H is a multiple of 512, otherwise they are stored by the lanes.
+  const bool bulk_scales = (scale_bytes % 16u) == 0u;
+  __shared__ int s_abort;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < s_in; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], uint32_t(cw));
+    }
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == cw) {
+    // ---- producer -------------------------------------------------------
+    if (lane == 0) {
+      int it = 0;
+      for (int64_t t = blockIdx.x; t < N; t += gridDim.x, ++it) {
+        const int s = it % s_in;
+        const uint32_t ph = uint32_t(it / s_in) & 1u;
+        if (it >= s_in && !mbar_wait_bounded(&empty[s], ph ^ 1u)) {
+          report(status, EP_DEV_TIMEOUT);
+          break;
+        }
+        mbar_arrive_expect_tx(&full[s], row_bytes);
+        bulk_g2s(in_base + size_t(s) * in_bytes, hidden + t * H, row_bytes, &full[s]);
+      }
+      // never leave the CTA with a load still writing its shared memory
+      for (int s = 0; s < s_in && s < it; ++s) {
+        const int last = it - 1 - ((it - 1 - s) % s_in);
+        if (!mbar_wait_bounded(&full[s], uint32_t(last / s_in) & 1u))
+          report(status, EP_DEV_TIMEOUT);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---- consumers --------------------------------------------------------
+    const bool issuer = (warp == 0 && lane == 0);
+    int it = 0;
+    for (int64_t t = blockIdx.x; t < N; t += gridDim.x, ++it) {
+      const int s = it % s_in;
+      const uint32_t ph = uint32_t(it / s_in) & 1u;
+      uint8_t* out = out_base + size_t(it % s_out) * out_bytes;
+      int p_l = -1;
+      float w_l = 0.0f;
+      if (lane < K) {
+        p_l = __ldg(pos + t * K + lane);
+        w_l = __ldg(w + t * K + lane);
+        if (p_l >= cap) {
+          report(status, EP_DEV_CAPACITY);
+          p_l = -1;
+        }
+      }
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait_bounded(&full[s], ph);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        if (lane == 0) report(status, EP_DEV_TIMEOUT);
+        s_abort = 1;
+      }
+      const uint8_t* row = in_base + size_t(s) * in_bytes;
+      for (int u = warp; u * kUnitCh < H; u += cw) {
+        const int c0 = u * kUnitCh + lane * 16;  // first channel of this lane
+        const bool act = c0 < H;                 // H % 128 == 0: whole groups
+        uint4 a = make_uint4(0u, 0u, 0u, 0u), b = a;
+        if (act && ok) {
+          a = *reinterpret_cast<const uint4*>(row + size_t(c0) * 2);
+          b = *reinterpret_cast<const uint4*>(row + size_t(c0) * 2 + 16);
+        }
+        float x[16];
+        float amax = unpack16(a, b, x);
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+        const float scale = __fdiv_rn(amax, 448.0f);
+        uint4 q = make_uint4(0u, 0u, 0u, 0u);
+        if (scale != 0.0f) q = quantize16(x, make_group_scale(scale));
+        if (act) {
+          *reinterpret_cast<uint4*>(out + c0) = q;
+          if (bulk_scales && (lane & 7) == 0)
+            reinterpret_cast<float*>(out + H)[c0 >> 7] = scale;
+        }
+        if (!bulk_scales) {
+          // lanes store their group's scale to every destination row
+          for (int k = 0; k < K; ++k) {
+            const int p = __shfl_sync(0xffffffffu, p_l, k);
+            if (act && (lane & 7) == 0 && p >= 0)
+              scales[int64_t(p) * G + (c0 >> 7)] = scale;
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (warp == 0 && lane < K && p_l >= 0 && recv_w) recv_w[p_l] = w_l;
+      // make this token's output stage visible to the bulk-copy engine
+      fence_proxy_async_smem();
+      // before the barrier: the stage the next token writes must have been
+      // read by its earlier stores (at most s_out - 2 groups left pending)
+      if (issuer) {
+        if (s_out >= 3)
+          bulk_wait_read<1>();
+        else
+          bulk_wait_read<0>();
+      }
+      named_barrier(1, cw * 32);
+      if (s_abort) break;
+      // lane 0 of warp 0 issues the stores; the positions reach it through a
+      // shuffle that the whole warp executes
+      if (warp == 0) {
+        for (int k = 0; k < K; ++k) {
+          const int p = __shfl_sync(0xffffffffu, p_l, k);
+          if (lane == 0 && p >= 0) {
+            bulk_s2g(recv + int64_t(p) * H, out, uint32_t(H));
+            if (bulk_scales)
+              bulk_s2g(scales + int64_t(p) * G, out + H, scale_bytes);
+          }
+        }
+        if (lane == 0) bulk_commit();
+      }
+    }
+    if (issuer) bulk_wait_all<0>();
+  }
+  __syncthreads();
+  zero_padding_rows<true>(row_src, offsets, E, H, cap, recv, scales, recv_w);
+}
+
+__global__ void k_debug_quantize(const float* __restrict__ x,
+                                 const float* __restrict__ scale,
+                                 uint8_t* __restrict__ out, int64_t n) {
+  // x is [n/16][16], scale one value per 16 values; exercises quantize16
+  const int64_t groups = n / 16;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < groups;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    float v[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = x[i * 16 + j];
+    const float s = scale[i];
+    uint4 q = make_uint4(0u, 0u, 0u, 0u);
+    if (s != 0.0f) q = quantize16(v, make_group_scale(s));
+    *reinterpret_cast<uint4*>(out + i * 16) = q;
+  }
+}
+
+struct Cfg {
   int threads = 0;
-  int stages = 0;
+  int s_in = 0;
+  int s_out = 0;
   size_t smem = 0;
 };
 
-DispatchCfg dispatch_cfg(int H) {
-  DispatchCfg c;
+Cfg fp8_cfg(int H) {
+  Cfg c;
   const int units = (H + kUnitCh - 1) / kUnitCh;
   const int cw = std::min(units, kMaxConsumerWarps);
   c.threads = (cw + 1) * 32;
-  const uint32_t stage_bytes = align128(uint32_t(H) * 2u);
-  c.stages = int(std::max<size_t>(2, std::min<size_t>(kMaxStages, kStageBudget / stage_bytes)));
-  c.smem = size_t(c.stages) * stage_bytes + 2 * kMaxStages * sizeof(uint64_t);
+  const uint32_t in_bytes = align128(uint32_t(H) * 2u);
+  const uint32_t out_bytes = align128(uint32_t(H) + uint32_t(H / 128) * 4u);
+  // ~100 KB per CTA so that two CTAs share an SM
+  c.s_in = int(std::max<size_t>(2, std::min<size_t>(4, (64 * 1024) / in_bytes)));
+  c.s_out = int(std::max<size_t>(2, std::min<size_t>(3, (36 * 1024) / out_bytes)));
+  c.smem = size_t(c.s_in) * in_bytes + size_t(c.s_out) * out_bytes +
+           2 * kMaxStages * sizeof(uint64_t);
+  return c;
+}
+
+Cfg bf16_cfg(int H) {
+  Cfg c;
+  c.threads = 32;
+  const uint32_t in_bytes = align128(uint32_t(H) * 2u);
+  c.s_in = int(std::max<size_t>(2, std::min<size_t>(kMaxStages, (72 * 1024) / in_bytes)));
+  c.smem = size_t(c.s_in) * in_bytes + kMaxStages * sizeof(uint64_t);
   return c;
 }
 
@@ -227,8 +451,9 @@ cudaError_t launch_dispatch(const void* hidden, const float* w,
                             int E, int H, int64_t cap, bool fp8, void* recv,
                             float* recv_scales, float* recv_w, int num_sms,
                             int32_t* status, cudaStream_t stream) {
-  const DispatchCfg c = dispatch_cfg(H);
-  auto kern = fp8 ? k_dispatch<true> : k_dispatch<false>;
+  const Cfg c = fp8 ? fp8_cfg(H) : bf16_cfg(H);
+  const void* kern = fp8 ? reinterpret_cast<const void*>(k_dispatch_fp8)
+                         : reinterpret_cast<const void*>(k_dispatch_bf16);
   cudaError_t err = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(c.smem));
   if (err != cudaSuccess) return err;
@@ -241,10 +466,25 @@ cudaError_t launch_dispatch(const void* hidden, const float* w,
   const int64_t grid = std::max<int64_t>(
       1, std::min<int64_t>(int64_t(num_sms) * per_sm,
                            std::max<int64_t>(N, (cap + 31) / 32)));
-  kern<<<int(grid), c.threads, c.smem, stream>>>(
-      static_cast<const uint16_t*>(hidden), w, pos, row_src, expert_offsets, N,
-      K, E, H, cap, static_cast<uint8_t*>(recv), recv_scales, recv_w, c.stages,
-      status);
+  const uint16_t* h = static_cast<const uint16_t*>(hidden);
+  uint8_t* r = static_cast<uint8_t*>(recv);
+  if (fp8)
+    k_dispatch_fp8<<<int(grid), c.threads, c.smem, stream>>>(
+        h, w, pos, row_src, expert_offsets, N, K, E, H, cap, r, recv_scales,
+        recv_w, c.s_in, c.s_out, status);
+  else
+    k_dispatch_bf16<<<int(grid), c.threads, c.smem, stream>>>(
+        h, w, pos, row_src, expert_offsets, N, K, E, H, cap, r, recv_w,
+        c.s_in, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_debug_quantize(const float* x, const float* scale,
+                                  uint8_t* out, int64_t n, cudaStream_t stream) {
+  const int64_t groups = n / 16;
+  if (groups == 0) return cudaSuccess;
+  const int grid = int(std::min<int64_t>((groups + 255) / 256, 148 * 16));
+  k_debug_quantize<<<grid, 256, 0, stream>>>(x, scale, out, n);
   return cudaGetLastError();
 }
 

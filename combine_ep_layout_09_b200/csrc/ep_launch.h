@@ -53,6 +53,8 @@ cudaError_t launch_prefetch(const int32_t* slot_expert, int R, int E, int B,
 
 cudaError_t launch_debug_e4m3(const float* x, uint8_t* out, int64_t n,
                              cudaStream_t stream);
+cudaError_t launch_debug_quantize(const float* x, const float* scale,
+                                  uint8_t* out, int64_t n, cudaStream_t stream);
 cudaError_t launch_debug_wait(const int32_t* flag, int64_t max_polls,
                               int32_t* status, cudaStream_t stream);
 

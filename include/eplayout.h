@@ -256,6 +256,13 @@ EP_API int ep_prefetch_weights(const int32_t* slot_expert, int R, int E, int B,
 EP_API int ep_debug_e4m3_encode(const float* x, uint8_t* out, int64_t n,
                          void* stream);
 
+/* out[i] = e4m3(RN(x[i] / group_scale[i/16])) for n values (n % 16 == 0),
+ * computed by the same device routine the FP8 dispatch quantises with
+ * (bracketed reciprocal products, correctly rounded division on the rare
+ * values near a rounding boundary); a zero scale gives code 0. */
+EP_API int ep_debug_quantize(const float* x, const float* group_scale,
+                             uint8_t* out, int64_t n, void* stream);
+
 /* One thread polls *flag until it is non-zero, giving up after `max_polls`
  * polls with EP_DEV_TIMEOUT OR-ed into *status: the bounded wait every
  * device-side spin in this library uses, exposed so its give-up path can be

@@ -68,6 +68,8 @@ def lib():
                                            i64, P, P]
         L.oracle_quantize_row.restype = None
         L.oracle_quantize_row.argtypes = [P, i32, P, P]
+        L.oracle_quantize_by_scale.restype = None
+        L.oracle_quantize_by_scale.argtypes = [P, P, i64, i32, P]
         L.oracle_dispatch_fp8.restype = None
         L.oracle_dispatch_fp8.argtypes = [P, P, P, P, P, i64, i32, i32, i32,
                                           i64, P, P, P]
@@ -183,6 +185,16 @@ def quantize_rows(rows: np.ndarray):
     for i in range(n):
         q[i], s[i] = quantize_row(rows[i])
     return q, s
+
+
+def quantize_by_scale(x: np.ndarray, scale: np.ndarray, group: int = 16):
+    """codes[i] = e4m3(fp32(x[i] / scale[i // group])), 0 where scale == 0."""
+    x = _c(x, np.float32).ravel()
+    scale = _c(scale, np.float32).ravel()
+    assert scale.size * group >= x.size
+    out = np.empty(x.size, np.uint8)
+    lib().oracle_quantize_by_scale(_p(x), _p(scale), x.size, group, _p(out))
+    return out
 
 
 def dispatch_fp8(hidden: np.ndarray, w: np.ndarray, lay: dict, E: int,

@@ -257,6 +257,23 @@ void oracle_quantize_row(const uint16_t* row, int H, uint8_t* q,
     }
 }
 
+/* Codes of values quantised by a given scale per group of `group` values:
+ * out[i] = e4m3(x[i] / scale[i / group]) with the quotient in fp32 (the
+ * inner step of oracle_quantize_row, for arbitrary scales); scale 0 gives
+ * code 0. */
+void oracle_quantize_by_scale(const float* x, const float* scale, int64_t n,
+                              int group, uint8_t* out) {
+    for (int64_t i = 0; i < n; ++i) {
+        float s = scale[i / group];
+        if (s == 0.0f) {
+            out[i] = 0;
+            continue;
+        }
+        float qf = x[i] / s;
+        out[i] = oracle_e4m3_encode(qf);
+    }
+}
+
 /* FP8 dispatch: each token row is quantised once and its codes and scales
  * copied to the K destination rows. Padding rows: zero codes, zero scales,
  * zero weight. recv_w may be NULL. */

@@ -41,3 +41,54 @@ def test_random_rest_and_specials():
                         np.float32)
     x = np.concatenate([x, specials])
     np.testing.assert_array_equal(gpu_encode(x), oracle.e4m3_encode(x))
+
+
+def gpu_quantize(x: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    xd = torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(DEV)
+    sd = torch.from_numpy(np.ascontiguousarray(scale, np.float32)).to(DEV)
+    out = torch.empty(x.size, dtype=torch.uint8, device=DEV)
+    ep.ep_debug_quantize(xd, sd, out)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+def _midpoints():
+    v = np.array([oracle.e4m3_decode(c)[0] for c in range(0x7F)])
+    return (v[:-1] + v[1:]) / 2
+
+
+def test_quantize_random_scales():
+    rng = np.random.default_rng(1)
+    G = 1 << 18
+    scale = np.exp2(rng.uniform(-130, 30, G)).astype(np.float32)
+    scale[::97] = 0.0
+    mag = np.exp2(rng.uniform(-12, 9.5, G * 16))
+    x = (np.repeat(scale.astype(np.float64), 16) * mag *
+         rng.choice([-1.0, 1.0], G * 16)).astype(np.float32)
+    x[::1001] = 0.0
+    x[5::1003] = -0.0
+    np.testing.assert_array_equal(gpu_quantize(x, scale),
+                                  oracle.quantize_by_scale(x, scale))
+
+
+def test_quantize_quotients_on_rounding_boundaries():
+    # x/s lands on, or one fp32 step either side of, every E4M3 midpoint, so
+    # the bracket disagrees and the correctly rounded division decides
+    rng = np.random.default_rng(2)
+    mids = _midpoints()
+    G = 1 << 16
+    scale = np.exp2(rng.uniform(-20, 20, G)).astype(np.float32)
+    m = rng.choice(mids, G * 16) * rng.choice([-1.0, 1.0], G * 16)
+    x = (np.repeat(scale.astype(np.float64), 16) * m).astype(np.float32)
+    nudge = rng.integers(-2, 3, G * 16)
+    x = np.nextafter(x, np.where(nudge > 0, np.inf, -np.inf).astype(
+        np.float32)) * (nudge != 0) + x * (nudge == 0)
+    x = x.astype(np.float32)
+    got = gpu_quantize(x, scale)
+    np.testing.assert_array_equal(got, oracle.quantize_by_scale(x, scale))
+    # exact ties with scale 1: the midpoints themselves
+    xm = np.concatenate([mids, -mids]).astype(np.float32)
+    xm = np.resize(xm, ((xm.size + 15) // 16) * 16)
+    sm = np.ones(xm.size // 16, np.float32)
+    np.testing.assert_array_equal(gpu_quantize(xm, sm),
+                                  oracle.quantize_by_scale(xm, sm))

@@ -152,3 +152,21 @@ def test_quantize_row_widths(H):
     rows = _bf16_rows(3, H, 8)
     q, s = oracle.quantize_rows(rows)
     assert q.shape == (3, H) and s.shape == (3, H // 128)
+
+
+def test_quantize_by_scale_matches_row_quantisation_and_library():
+    rows = _bf16_rows(6, 512, 11)
+    q, s = oracle.quantize_rows(rows)
+    x = (rows.astype(np.uint32) << 16).view(np.float32)
+    got = oracle.quantize_by_scale(x, s, group=128).reshape(6, 512)
+    np.testing.assert_array_equal(got, q)
+    rng = np.random.default_rng(12)
+    xs = (rng.standard_normal(4096) * 10).astype(np.float32)
+    sc = np.exp2(rng.uniform(-20, 20, 256)).astype(np.float32)
+    sc[3] = 0.0
+    got = oracle.quantize_by_scale(xs, sc, group=16)
+    quot = (xs / np.repeat(sc, 16)).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        ref = torch_e4m3(np.clip(quot, -448, 448))
+    ref[48:64] = 0
+    np.testing.assert_array_equal(got, ref)
