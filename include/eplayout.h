@@ -124,7 +124,7 @@ EP_API int ep_layout(const int32_t* topk_experts, int R, int S, int K, int E,
  * on a GPU until the process exits. Nothing is allocated by the call.
  *   - Limit: problems with ep_layout_workspace_bytes(R*S, K, E) larger than
  *     EP_LAYOUT_STATIC_SCRATCH_BYTES are refused with EP_ERR_WORKSPACE
- *     before any CUDA call (E=256 fits up to about 4.2 M entries N*K).
+ *     before any CUDA call (E=256 fits up to about 16 M entries N*K).
  *   - The first call on each GPU looks up the array's device address
  *     (cudaGetSymbolAddress, with that GPU current) and caches it; make that
  *     first call before any stream capture.

@@ -21,6 +21,7 @@ def compare(topk, R, S, E, pad, cap=None):
     np.testing.assert_array_equal(g["pos"], o["pos"])
     np.testing.assert_array_equal(g["row_src"], o["row_src"])
     assert bool(g["status"] & 1) == bool(o["status"] & oracle.ST_BAD_EXPERT)
+    assert g["status"] & ~1 == 0      # no timeout, no capacity error
     return g, o
 
 
@@ -109,3 +110,25 @@ def test_repeat_calls_reuse_workspace():
     a = gpu_layout(topk, 8, 512, 32, 1)
     b = gpu_layout(topk, 8, 512, 32, 1)
     np.testing.assert_array_equal(a["pos"], b["pos"])
+
+
+@pytest.mark.parametrize("E,pad", [(256, 1), (64, 128)])
+def test_large_input_takes_two_kernel_path(E, pad):
+    # 3 M entries: more 4096-entry tiles than can be co-resident, so the
+    # histogram + look-back scan pair runs instead of the fused kernel
+    R, S, K = 8, 49152, 8
+    rng = np.random.default_rng(E + pad)
+    topk = rng.integers(0, E, size=(R * S, K)).astype(np.int32)
+    compare(topk, R, S, E, pad)
+
+
+@pytest.mark.parametrize("E", [2, 96, 128, 192, 256, 320, 512, 768])
+def test_expert_counts_across_thread_mappings(E):
+    # E values that map experts to threads differently (pairs of look-back
+    # threads, chunks of warps per expert), with several tiles
+    R = 2 if E % 2 == 0 else 1
+    rng = np.random.default_rng(E)
+    S = 9000 // R
+    topk = rng.integers(0, E, size=(R * S, 8)).astype(np.int32)
+    g, _ = compare(topk, R, S, E, 4)
+    assert g["status"] == 0

@@ -83,7 +83,7 @@ def test_static_scratch_matches_workspace_entry_point(first, second):
 def test_static_scratch_refuses_problems_beyond_its_size():
     f = _static_fn()
     R, K, E = 8, 8, 1024
-    S = 64 * 1024                      # needs far more than 1 MiB of scratch
+    S = 256 * 1024                     # needs far more than 1 MiB of scratch
     assert ep.ep_layout_workspace_bytes(R * S, K, E) > SCRATCH_BYTES
     dummy = torch.zeros(16, dtype=torch.int32, device=DEV)
     p = dummy.data_ptr()
