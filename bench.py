@@ -95,6 +95,24 @@ def dist_info():
     return ws, rank, local
 
 
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank time over all ranks (identity without a group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    if dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def total_value_gbs(bytes_per_step: int, steps: int, world: int,
+                    ms_max: float) -> float:
+    """Whole-job throughput: bytes of all steps on all ranks / max time."""
+    return bytes_per_step * steps * world / (ms_max * 1e-3) / 1e9
+
+
 class ClockSampler:
     """Samples SM clock and throttle reasons with NVML every 10 ms."""
 
@@ -255,22 +273,12 @@ class Path:
         self.ep.ep_combine(self.y, self.pos, self.w, wl.N, wl.K, wl.H,
                            self.out, status=self.status, cap=self.cap)
 
-    def step(self, ev=None):
-        if ev is not None:
-            ev[0].record()
+    def step(self):
         self.layout()
-        if ev is not None:
-            ev[1].record()
         if self.wl.B > 0:
             self.plan_prefetch()
-        if ev is not None:
-            ev[2].record()
         self.dispatch()
-        if ev is not None:
-            ev[3].record()
         self.combine()
-        if ev is not None:
-            ev[4].record()
 
 
 def run_gpu(args, wl):
@@ -288,13 +296,8 @@ def run_gpu(args, wl):
             import torch.distributed as dist
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if ws == 1:
-            return x
-        import torch.distributed as dist
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def rank_max(x: float) -> float:
+        return max_over_ranks(x, dev)
 
     path = Path(wl, dev, seed_offset=rank)
     torch.cuda.synchronize()
@@ -314,30 +317,57 @@ def run_gpu(args, wl):
     b_pre = bytes_prefetch(n_slots, wl.H, wl.I) if wl.B else 0
     b_step = b_lay + b_dis + b_com + b_pre
 
+    # The K timed steps are captured once into a CUDA graph (the library is
+    # capture-safe: no allocation, no synchronisation) and replayed once, so
+    # no host launch gap sits between kernels. Each kernel's own average is
+    # then timed the same way, from a graph of K launches of that kernel
+    # alone (events between kernels inside one graph would add their own
+    # gaps to the kernels they bracket).
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)]
-           for _ in range(K)]
+
+    def capture(fn, n):
+        cs = torch.cuda.Stream()
+        cs.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cs):
+            for _ in range(n):
+                fn()
+        torch.cuda.synchronize()
+        return g
+
+    def replay_ms(g):
+        a_, b_ = (torch.cuda.Event(enable_timing=True),
+                  torch.cuda.Event(enable_timing=True))
+        a_.record()
+        g.replay()
+        b_.record()
+        torch.cuda.synchronize()
+        return a_.elapsed_time(b_)
+
+    graph = capture(path.step, K)
     start = torch.cuda.Event(enable_timing=True)
     stop = torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         start.record()
-        for i in range(K):
-            path.step(evs[i])
+        graph.replay()
         stop.record()
         torch.cuda.synchronize()
     barrier()
+    del graph
+    parts = {"layout": path.layout, "dispatch": path.dispatch,
+             "combine": path.combine}
+    if wl.B > 0:
+        parts["plan_prefetch"] = path.plan_prefetch
+    avg = {"plan_prefetch": 0.0}
+    for name, fn in parts.items():
+        g = capture(fn, K)
+        avg[name] = replay_ms(g) / K * 1e3     # us per launch
+        del g
+    med = avg
     ms = start.elapsed_time(stop)
-    ms_max = max_over_ranks(ms)
-    per = {"layout": [], "plan_prefetch": [], "dispatch": [], "combine": []}
-    for e in evs:
-        per["layout"].append(e[0].elapsed_time(e[1]))
-        per["plan_prefetch"].append(e[1].elapsed_time(e[2]))
-        per["dispatch"].append(e[2].elapsed_time(e[3]))
-        per["combine"].append(e[3].elapsed_time(e[4]))
-    med = {k: statistics.median(v) * 1e3 for k, v in per.items()}   # us
-    avg = {k: statistics.fmean(v) * 1e3 for k, v in per.items()}
+    ms_max = rank_max(ms)
     st = int(path.status[0].item())
     if st:
         raise RuntimeError(f"device status after timing: {st}")
@@ -345,12 +375,12 @@ def run_gpu(args, wl):
     # ---- end to end: host buffers in, host result out, every step -------
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, path, b_step, max_over_ranks, barrier)
+        e2e = run_e2e(args, path, b_step, rank_max, barrier)
 
     result = None
     if rank == 0:
         peak, peak_src = measured_peak()
-        value = b_step * K * ws / (ms_max * 1e-3) / 1e9
+        value = total_value_gbs(b_step, K, ws, ms_max)
         comb_gbs = b_com / (avg["combine"] * 1e-6) / 1e9
         dis_gbs = b_dis / (avg["dispatch"] * 1e-6) / 1e9
         dom = "combine" if avg["combine"] >= avg["dispatch"] else "dispatch"
@@ -384,6 +414,9 @@ def run_gpu(args, wl):
                 "l2": "no flush: every step moves >4 GB, inputs larger "
                       "than the 126 MB L2",
                 "parallelism": f"{ws} independent replica(s), one per GPU",
+                "timing": "K steps captured in one CUDA graph, replayed "
+                          "once, CUDA events around the replay; per-kernel "
+                          "times from a graph of K launches of that kernel",
             },
             "breakdown": {
                 "layout_us": round(med["layout"], 2),
@@ -527,7 +560,7 @@ def run_reference(args, wl):
         return None
     # about a minute of oracle work for the whole warm-up + timed run
     per_tok = 0.8e-3
-    n_tok = int(max(1, min(4096, 60.0 / (args.steps + args.warmup) /
+    n_tok = int(max(1, min(4096, wl.N, 60.0 / (args.steps + args.warmup) /
                            per_tok)))
     topk, w, h, y = oracle_sample(wl, n_tok)
     for _ in range(args.warmup):
