@@ -7,10 +7,17 @@
 // one fused multiply-add per k, k ascending from +0, then rounded to bf16
 // (nearest even), so the result is a fixed function of its inputs.
 //
-// Persistent CTAs walk tokens; the threads of a CTA split the row into
-// 16-byte vectors (8 channels). Each thread issues its K gathered loads
-// before any arithmetic, so K * 16 bytes per thread are in flight. The kernel
-// reads K rows per written row: it is bound by HBM read bandwidth.
+// The kernel reads K rows per written row: it is bound by HBM read bandwidth.
+// Two forms:
+//   k_combine_tma  (large batches) persistent, one CTA per SM: a producer
+//                  warp bulk-loads the K gathered part-rows of a (token, part)
+//                  unit into a shared-memory stage (three stages, ~170 KB of
+//                  reads in flight per SM); consumer threads reduce from
+//                  shared memory; one thread bulk-stores the output part.
+//   k_combine<K>   (small batches) CTAs walk tokens, threads split the row
+//                  into 16-byte vectors and issue their K gathered loads
+//                  before any arithmetic.
+// Both run the same fma chain in the same k order.
 #include <algorithm>
 
 #include "ep_device.cuh"
@@ -105,6 +112,193 @@ __global__ void __launch_bounds__(kCombineMaxThreads)
   }
 }
 
+// ---------------------------------------------------------------------------
+// TMA-fed combine: a producer warp bulk-loads, for each (token, row part),
+// the K gathered part-rows into a shared-memory stage; consumer threads run
+// the fma chain from shared memory and one thread bulk-stores the output
+// part. Three stages keep ~170 KB of reads in flight per SM.
+// ---------------------------------------------------------------------------
+
+constexpr int kTmaMaxConsumerWarps = 16;
+constexpr int kTmaStages = 3;
+constexpr int kTmaOutStages = 2;
+constexpr uint32_t kTmaStageTarget = 64 * 1024;  // K part-rows per stage
+
+__host__ __device__ constexpr uint32_t al128(uint32_t x) { return (x + 127u) & ~127u; }
+
+struct TmaShape {
+  int part_ch;   // channels per part (multiple of 8)
+  int parts;     // parts per row
+  int cw;        // consumer warps
+  uint32_t in_bytes, out_bytes;
+  size_t smem;
+};
+
+__host__ __device__ inline TmaShape tma_shape(int H, int K) {
+  TmaShape sh;
+  int max_ch = int(kTmaStageTarget / (uint32_t(K) * 2u)) & ~7;
+  if (max_ch < 8) max_ch = 8;
+  sh.parts = (H + max_ch - 1) / max_ch;
+  sh.part_ch = ((H + sh.parts - 1) / sh.parts + 7) & ~7;
+  const int part_v = sh.part_ch / 8;
+  int cw = (part_v + 31) / 32;
+  sh.cw = cw < kTmaMaxConsumerWarps ? cw : kTmaMaxConsumerWarps;
+  sh.in_bytes = al128(uint32_t(K) * uint32_t(sh.part_ch) * 2u);
+  sh.out_bytes = al128(uint32_t(sh.part_ch) * 2u);
+  // stages, output stages, then per stage: full / empty barriers, mask, weights
+  sh.smem = size_t(kTmaStages) * sh.in_bytes + size_t(kTmaOutStages) * sh.out_bytes +
+            size_t(kTmaStages) * (16 + 4 + 4 * 32) + 64;
+  return sh;
+}
+
+__global__ void __launch_bounds__((kTmaMaxConsumerWarps + 1) * 32, 1)
+    k_combine_tma(const uint16_t* __restrict__ y, const int32_t* __restrict__ pos,
+                  const float* __restrict__ w, int64_t N, int K, int H,
+                  int64_t cap, uint16_t* __restrict__ out,
+                  int32_t* __restrict__ status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const TmaShape sh = tma_shape(H, K);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cw = sh.cw;
+  uint8_t* in_base = smem;
+  uint8_t* out_base = smem + size_t(kTmaStages) * sh.in_bytes;
+  uint8_t* meta = out_base + size_t(kTmaOutStages) * sh.out_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(meta);
+  uint64_t* empty = full + kTmaStages;
+  uint32_t* vmask = reinterpret_cast<uint32_t*>(empty + kTmaStages);
+  float* wk = reinterpret_cast<float*>(vmask + kTmaStages);  // [stages][32]
+  __shared__ int s_abort;
+  const int64_t units = N * sh.parts;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTmaStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], uint32_t(cw));
+    }
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == cw) {
+    // ---- producer warp: lane k handles the k-th gathered part-row --------
+    int it = 0;
+    int64_t u = blockIdx.x;
+    int p_n = -1;
+    float w_n = 0.0f;
+    if (u < units && lane < K) {
+      const int64_t t0 = u / sh.parts;
+      p_n = __ldg(pos + t0 * K + lane);
+      w_n = __ldg(w + t0 * K + lane);
+    }
+    for (; u < units; u += gridDim.x, ++it) {
+      const int64_t t = u / sh.parts;
+      const int part = int(u - t * sh.parts);
+      const int c0 = part * sh.part_ch;
+      const int len = min(sh.part_ch, H - c0);
+      const uint32_t bytes = uint32_t(len) * 2u;
+      const int p = p_n;
+      const float wv = w_n;
+      {  // positions of the next unit, one unit ahead
+        const int64_t un = u + gridDim.x;
+        if (un < units && lane < K) {
+          const int64_t tn = un / sh.parts;
+          p_n = __ldg(pos + tn * K + lane);
+          w_n = __ldg(w + tn * K + lane);
+        }
+      }
+      const bool valid = lane < K && p >= 0 && p < cap;
+      if (lane < K && p >= cap) report(status, EP_DEV_CAPACITY);
+      const unsigned m = __ballot_sync(0xffffffffu, valid);
+      const int s = it % kTmaStages;
+      const uint32_t ph = uint32_t(it / kTmaStages) & 1u;
+      bool ok = true;
+      if (lane == 0 && it >= kTmaStages) ok = mbar_wait_bounded(&empty[s], ph ^ 1u);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        if (lane == 0) report(status, EP_DEV_TIMEOUT);
+        break;
+      }
+      if (lane < 32) wk[s * 32 + lane] = wv;
+      if (lane == 0) {
+        vmask[s] = m;
+        mbar_arrive_expect_tx(&full[s], uint32_t(__popc(m)) * bytes);
+      }
+      __syncwarp();
+      if (valid)
+        bulk_g2s(in_base + size_t(s) * sh.in_bytes + size_t(lane) * sh.part_ch * 2,
+                 y + int64_t(p) * H + c0, bytes, &full[s]);
+    }
+    // never leave with a load still writing shared memory
+    if (lane == 0)
+      for (int s = 0; s < kTmaStages && s < it; ++s) {
+        const int last = it - 1 - ((it - 1 - s) % kTmaStages);
+        if (!mbar_wait_bounded(&full[s], uint32_t(last / kTmaStages) & 1u))
+          report(status, EP_DEV_TIMEOUT);
+      }
+    __syncwarp();
+  } else {
+    // ---- consumers --------------------------------------------------------
+    const bool issuer = (warp == 0 && lane == 0);
+    const int nthreads = cw * 32;
+    int it = 0;
+    for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++it) {
+      const int64_t t = u / sh.parts;
+      const int part = int(u - t * sh.parts);
+      const int c0 = part * sh.part_ch;
+      const int len = min(sh.part_ch, H - c0);
+      const int s = it % kTmaStages;
+      const uint32_t ph = uint32_t(it / kTmaStages) & 1u;
+      uint8_t* ob = out_base + size_t(it % kTmaOutStages) * sh.out_bytes;
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait_bounded(&full[s], ph);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        if (lane == 0) report(status, EP_DEV_TIMEOUT);
+        s_abort = 1;
+      }
+      const uint32_t m = vmask[s];
+      const uint8_t* st = in_base + size_t(s) * sh.in_bytes;
+      for (int v = threadIdx.x; v < (len >> 3); v += nthreads) {
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int k = 0; k < K; ++k) {
+          if (!((m >> k) & 1u)) continue;
+          const uint4 d = *reinterpret_cast<const uint4*>(st + size_t(k) * sh.part_ch * 2 +
+                                                          size_t(v) * 16);
+          fma8(acc, wk[s * 32 + k], d);
+        }
+        *reinterpret_cast<uint4*>(ob + size_t(v) * 16) = pack8(acc);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      fence_proxy_async_smem();
+      // the other output stage must have been read by its store
+      if (issuer) bulk_wait_read<0>();
+      asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+      if (s_abort) break;
+      if (issuer) {
+        bulk_s2g(out + t * H + c0, ob, uint32_t(len) * 2u);
+        bulk_commit();
+      }
+    }
+    if (issuer) bulk_wait_all<0>();
+  }
+}
+
+cudaError_t run_tma(const uint16_t* y, const int32_t* pos, const float* w,
+                    int64_t N, int K, int H, int64_t cap, uint16_t* out,
+                    int num_sms, int32_t* status, cudaStream_t stream) {
+  const TmaShape sh = tma_shape(H, K);
+  cudaError_t err = cudaFuncSetAttribute(
+      k_combine_tma, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sh.smem));
+  if (err != cudaSuccess) return err;
+  const int64_t units = N * sh.parts;
+  const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(units, num_sms));
+  k_combine_tma<<<int(grid), (sh.cw + 1) * 32, sh.smem, stream>>>(
+      y, pos, w, N, K, H, cap, out, status);
+  return cudaGetLastError();
+}
+
 template <int KT>
 cudaError_t run(const uint16_t* y, const int32_t* pos, const float* w,
                 int64_t N, int K, int H, int64_t cap, uint16_t* out,
@@ -133,6 +327,11 @@ cudaError_t launch_combine(const void* y_, const int32_t* pos, const float* w,
                            int num_sms, int32_t* status, cudaStream_t stream) {
   const uint16_t* y = static_cast<const uint16_t*>(y_);
   uint16_t* out = static_cast<uint16_t*>(out_);
+  // The TMA pipeline needs enough (token, part) units per SM to fill its
+  // stages; small batches (decode) are faster with the register gather.
+  const TmaShape sh = tma_shape(H, K);
+  if (sh.smem <= 200 * 1024 && N * sh.parts >= 16 * int64_t(num_sms))
+    return run_tma(y, pos, w, N, K, H, cap, out, num_sms, status, stream);
   switch (K) {
     case 1: return run<1>(y, pos, w, N, K, H, cap, out, num_sms, status, stream);
     case 2: return run<2>(y, pos, w, N, K, H, cap, out, num_sms, status, stream);
