@@ -8,6 +8,10 @@
 // buffer whose rows [0, E) are all experts and whose later rows are the
 // local prefetch slots filled by prefetch_weight.
 //
+// Prefetch: k_prefetch_tma streams the used slots through bulk copies (one
+// 16 KB chunk per unit); k_prefetch (16-byte vector copies) serves slot
+// tables too large to compact in shared memory.
+//
 // Plan: the unpadded expert-grouped rows (experts in order) are cut into R
 // chunks of T = S*K rows. Expert e holds rows [C_e, C_e + c_e); it meets
 // chunks p = floor(C_e/T) .. q = floor((C_e + c_e - 1)/T). Chunk p reads
@@ -174,6 +178,92 @@ __global__ void __launch_bounds__(kCopyThreads)
   }
 }
 
+// TMA form of the slot copy: one-warp CTAs first compact the used slots into
+// shared memory, then stream their (slot, projection, chunk) units through a
+// ring of bulk loads and bulk stores (no data passes through registers).
+constexpr int kTmaChunk = 16384;   // bytes per unit
+constexpr int kTmaCopyStages = 4;
+constexpr int kMaxSlotList = 1024;
+
+__global__ void __launch_bounds__(32)
+    k_prefetch_tma(const int32_t* __restrict__ slot_expert, int RB, int E,
+                   int64_t row_bytes, uint8_t* __restrict__ gate,
+                   uint8_t* __restrict__ up, uint8_t* __restrict__ down) {
+  extern __shared__ __align__(128) uint8_t smb[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smb + kTmaCopyStages * kTmaChunk);
+  int32_t* list = reinterpret_cast<int32_t*>(full + kTmaCopyStages);  // (slot, e)
+  __shared__ int s_n;
+  const int lane = threadIdx.x;
+  // compact the used slots, in slot order
+  int n = 0;
+  for (int b = 0; b < RB; b += 32) {
+    const int slot = b + lane;
+    const int32_t e = slot < RB ? __ldg(slot_expert + slot) : -1;
+    const bool used = e >= 0 && e < E;
+    const unsigned m = __ballot_sync(0xffffffffu, used);
+    if (used) {
+      const int at = n + __popc(m & ((1u << lane) - 1u));
+      list[2 * at] = slot;
+      list[2 * at + 1] = e;
+    }
+    n += __popc(m);
+  }
+  if (lane == 0) s_n = n;
+  __syncwarp();
+  const int64_t nchunk = (row_bytes + kTmaChunk - 1) / kTmaChunk;
+  const int64_t units = int64_t(s_n) * 3 * nchunk;
+  const int64_t first = blockIdx.x, stride = gridDim.x;
+  const int64_t n_mine = first < units ? (units - 1 - first) / stride + 1 : 0;
+  if (lane != 0 || n_mine == 0) return;
+
+  auto unit = [&](int64_t i, const uint8_t** src, uint8_t** dst, uint32_t* bytes) {
+    const int64_t u = first + i * stride;
+    const int64_t j = u / (3 * nchunk);
+    const int64_t rem = u - j * 3 * nchunk;
+    const int proj = int(rem / nchunk);
+    const int64_t ch = rem - int64_t(proj) * nchunk;
+    uint8_t* W = proj == 0 ? gate : (proj == 1 ? up : down);
+    const int64_t off = ch * kTmaChunk;
+    *bytes = uint32_t(min(int64_t(kTmaChunk), row_bytes - off));
+    *src = W + int64_t(list[2 * j + 1]) * row_bytes + off;
+    *dst = W + (int64_t(E) + list[2 * j]) * row_bytes + off;
+  };
+  for (int s = 0; s < kTmaCopyStages; ++s) mbar_init(&full[s], 1);
+  fence_mbar_init();
+  for (int64_t i = 0; i < kTmaCopyStages && i < n_mine; ++i) {
+    const uint8_t* src;
+    uint8_t* dst;
+    uint32_t bytes;
+    unit(i, &src, &dst, &bytes);
+    mbar_arrive_expect_tx(&full[i], bytes);
+    bulk_g2s(smb + size_t(i) * kTmaChunk, src, bytes, &full[i]);
+  }
+  for (int64_t i = 0; i < n_mine; ++i) {
+    const int s = int(i % kTmaCopyStages);
+    const uint8_t* src;
+    uint8_t* dst;
+    uint32_t bytes;
+    unit(i, &src, &dst, &bytes);
+    if (!mbar_wait_bounded(&full[s], uint32_t(i / kTmaCopyStages) & 1u)) break;
+    bulk_s2g(dst, smb + size_t(s) * kTmaChunk, bytes);
+    bulk_commit();
+    const int64_t nxt = i - 1 + kTmaCopyStages;
+    if (i >= 1 && nxt < n_mine) {
+      const int sp = int((i - 1) % kTmaCopyStages);
+      bulk_wait_read<1>();
+      unit(nxt, &src, &dst, &bytes);
+      mbar_arrive_expect_tx(&full[sp], bytes);
+      bulk_g2s(smb + size_t(sp) * kTmaChunk, src, bytes, &full[sp]);
+    }
+  }
+  // drain: loads in flight after a give-up, then every store
+  for (int64_t i = 0; i < kTmaCopyStages && i < n_mine; ++i) {
+    const int64_t last = n_mine - 1 - ((n_mine - 1 - i) % kTmaCopyStages);
+    mbar_wait_bounded(&full[i], uint32_t(last / kTmaCopyStages) & 1u);
+  }
+  bulk_wait_all<0>();
+}
+
 __global__ void k_debug_e4m3(const float* __restrict__ x, uint8_t* __restrict__ out,
                              int64_t n) {
   const int64_t pairs = (n + 1) / 2;
@@ -220,10 +310,27 @@ cudaError_t launch_plan_balanced(const int32_t* counts, int R, int S, int K,
 cudaError_t launch_prefetch(const int32_t* slot_expert, int R, int E, int B,
                             int64_t elems, void* gate, void* up, void* down,
                             int num_sms, cudaStream_t stream) {
+  const int64_t RB = int64_t(R) * B;
+  if (RB == 0 || elems == 0) return cudaSuccess;
+  if (RB <= kMaxSlotList) {
+    const size_t smem = size_t(kTmaCopyStages) * kTmaChunk +
+                        kTmaCopyStages * sizeof(uint64_t) + 2 * kMaxSlotList * 4;
+    cudaError_t err = cudaFuncSetAttribute(
+        k_prefetch_tma, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (err != cudaSuccess) return err;
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_prefetch_tma, 32,
+                                                        smem);
+    if (err != cudaSuccess) return err;
+    const int grid = num_sms * std::max(1, per_sm);
+    k_prefetch_tma<<<grid, 32, smem, stream>>>(
+        slot_expert, int(RB), E, elems * 2, static_cast<uint8_t*>(gate),
+        static_cast<uint8_t*>(up), static_cast<uint8_t*>(down));
+    return cudaGetLastError();
+  }
   const int64_t vecs = elems * 2 / 16;
   const int64_t nchunk = (vecs + kCopyVec - 1) / kCopyVec;
-  const int64_t units = int64_t(R) * B * 3 * nchunk;
-  if (units == 0) return cudaSuccess;
+  const int64_t units = RB * 3 * nchunk;
   int per_sm = 0;
   cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
       &per_sm, k_prefetch, kCopyThreads, 0);
@@ -231,7 +338,7 @@ cudaError_t launch_prefetch(const int32_t* slot_expert, int R, int E, int B,
   const int64_t grid = std::max<int64_t>(
       1, std::min<int64_t>(units, int64_t(num_sms) * std::max(1, per_sm)));
   k_prefetch<<<int(grid), kCopyThreads, 0, stream>>>(
-      slot_expert, R * B, E, vecs, static_cast<uint4*>(gate),
+      slot_expert, int(RB), E, vecs, static_cast<uint4*>(gate),
       static_cast<uint4*>(up), static_cast<uint4*>(down));
   return cudaGetLastError();
 }

@@ -124,3 +124,22 @@ def test_prefetch_balanced_full_size():
                 else:
                     assert after[r] == b[r]
         assert torch.equal(after[:w.E], b[:w.E])
+
+
+@pytest.mark.parametrize("R,B,E,shape", [
+    (8, 4, 256, (3, 5000)),      # chunked copy, last chunk shorter
+    (64, 20, 128, (2, 40)),      # more slots than the compacted list holds
+])
+def test_prefetch_forms_against_oracle(R, B, E, shape):
+    rng = np.random.default_rng(R * B)
+    rows = E + R * B
+    W = [rng.integers(0, 65535, size=(rows, *shape), dtype=np.uint16)
+         for _ in range(3)]
+    slots = rng.integers(-1, E, size=(R, B)).astype(np.int32)
+    slots[rng.random(slots.shape) < 0.5] = -1
+    dev = [to_dev(x.view(np.int16)).view(torch.bfloat16) for x in W]
+    ep.ep_prefetch_weights(to_dev(slots), R, E, B, *dev)
+    torch.cuda.synchronize()
+    for x, d in zip(W, dev):
+        got = d.view(torch.int16).cpu().numpy().view(np.uint16)
+        np.testing.assert_array_equal(got, oracle.prefetch(slots, E, x))
