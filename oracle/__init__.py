@@ -20,6 +20,13 @@ Parity status of each function (what pins it, in tests/test_oracle_*.py):
   plan_balanced                           brute-force row-by-row planner,
                                           every rank exactly S*K rows
   prefetch                                slot rows equal source rows
+  dispatch_backward                       adjoint of bf16 dispatch (fp64
+                                          inner products), brute force
+  combine_backward_rows / _weights        adjoint of combine, finite
+                                          differences of combine_f64 in w,
+                                          numpy einsum in fp64
+  gather_row_values                       closed form, round trip with
+                                          dispatch's recv_w
 """
 from __future__ import annotations
 
@@ -77,6 +84,16 @@ def lib():
         L.oracle_combine.argtypes = [P, P, P, i64, i32, i32, i64, P]
         L.oracle_combine_f64.restype = None
         L.oracle_combine_f64.argtypes = [P, P, P, i64, i32, i32, i64, P]
+        L.oracle_dispatch_backward.restype = None
+        L.oracle_dispatch_backward.argtypes = [P, P, i64, i32, i32, i64, P]
+        L.oracle_combine_backward_rows.restype = None
+        L.oracle_combine_backward_rows.argtypes = [P, P, P, P, P, i64, i32,
+                                                   i32, i32, i64, P]
+        L.oracle_combine_backward_weights.restype = None
+        L.oracle_combine_backward_weights.argtypes = [P, P, P, i64, i32, i32,
+                                                      i64, P]
+        L.oracle_gather_row_values.restype = None
+        L.oracle_gather_row_values.argtypes = [P, P, i64, i32, i64, P]
         L.oracle_plan_balanced.restype = i32
         L.oracle_plan_balanced.argtypes = [P, i32, i32, i32, i32, i32, P, P,
                                            P, P, P]
@@ -237,6 +254,58 @@ def combine_f64(y: np.ndarray, pos: np.ndarray, w: np.ndarray) -> np.ndarray:
     N, K = pos.shape
     out = np.empty((N, H), np.float64)
     lib().oracle_combine_f64(_p(y), _p(pos), _p(w), N, K, H, cap, _p(out))
+    return out
+
+
+# --- backward pair ----------------------------------------------------------
+
+def dispatch_backward(grad_recv: np.ndarray, pos: np.ndarray) -> np.ndarray:
+    """grad_hidden [N,H] bf16 bits: sum over k of the receive-row grads."""
+    g = _c(grad_recv, np.uint16)
+    pos = _c(pos, np.int32)
+    cap, H = g.shape
+    N, K = pos.shape
+    out = np.empty((N, H), np.uint16)
+    lib().oracle_dispatch_backward(_p(g), _p(pos), N, K, H, cap, _p(out))
+    return out
+
+
+def combine_backward_rows(grad_out: np.ndarray, w: np.ndarray, lay: dict,
+                          E: int, cap: int, fill: int = 0x7FBF) -> np.ndarray:
+    """grad of the expert outputs [cap,H] bf16 bits (untouched rows keep
+    `fill`)."""
+    g = _c(grad_out, np.uint16)
+    w = _c(w, np.float32)
+    N, H = g.shape
+    K = lay["pos"].shape[1]
+    out = np.full((cap, H), fill, np.uint16)
+    lib().oracle_combine_backward_rows(
+        _p(g), _p(w), _p(_c(lay["pos"], np.int32)),
+        _p(_c(lay["row_src"], np.int32)), _p(_c(lay["offsets"], np.int32)),
+        N, K, E, H, cap, _p(out))
+    return out
+
+
+def combine_backward_weights(grad_out: np.ndarray, y: np.ndarray,
+                             pos: np.ndarray) -> np.ndarray:
+    """grad of the route weights [N,K], in double precision."""
+    g = _c(grad_out, np.uint16)
+    y = _c(y, np.uint16)
+    pos = _c(pos, np.int32)
+    N, H = g.shape
+    K = pos.shape[1]
+    out = np.empty((N, K), np.float64)
+    lib().oracle_combine_backward_weights(_p(g), _p(y), _p(pos), N, K, H,
+                                          y.shape[0], _p(out))
+    return out
+
+
+def gather_row_values(row_vals: np.ndarray, pos: np.ndarray) -> np.ndarray:
+    v = _c(row_vals, np.float32)
+    pos = _c(pos, np.int32)
+    N, K = pos.shape
+    out = np.empty((N, K), np.float32)
+    lib().oracle_gather_row_values(_p(v), _p(pos), N, K, v.shape[0], _p(out))
     return out
 
 

@@ -423,3 +423,80 @@ void oracle_prefetch(const int32_t* slot_expert, int R, int E, int B,
                 W[dst * elems + i] = W[(int64_t)e * elems + i];
         }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Backward pair [DEP "DeepEP介绍": kernels for training; MEP "快速上手":    */
+/* combine returns gathered_route_weights_sk for the backward pass]          */
+/* ------------------------------------------------------------------------ */
+
+/* Dispatch backward (bf16 dispatch): each token's gradient is the sum of the
+ * gradients of its K receive rows, in fp32, k = 0..K-1 from +0, rounded to
+ * bf16. This is combine with every weight equal to one. */
+void oracle_dispatch_backward(const uint16_t* grad_recv, const int32_t* pos,
+                              int64_t N, int K, int H, int64_t cap,
+                              uint16_t* grad_hidden) {
+    for (int64_t t = 0; t < N; ++t)
+        for (int h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int k = 0; k < K; ++k) {
+                int32_t p = pos[t * K + k];
+                if (p < 0 || p >= cap) continue;
+                acc = acc + oracle_bf16_to_f32(grad_recv[(int64_t)p * H + h]);
+            }
+            grad_hidden[t * H + h] = oracle_f32_to_bf16(acc);
+        }
+}
+
+/* Combine backward, expert-output side: the gradient of receive row
+ * pos[t,k] is w[t,k] * grad_out[t], the product in fp32 rounded to bf16.
+ * Padding rows (row_src == -1 below offsets[E]) get zeros; rows at and above
+ * offsets[E] are not touched. */
+void oracle_combine_backward_rows(const uint16_t* grad_out, const float* w,
+                                  const int32_t* pos, const int32_t* row_src,
+                                  const int32_t* offsets, int64_t N, int K,
+                                  int E, int H, int64_t cap,
+                                  uint16_t* grad_rows) {
+    for (int64_t r = 0; r < offsets[E] && r < cap; ++r)
+        if (row_src[r] < 0)
+            for (int h = 0; h < H; ++h) grad_rows[r * H + h] = 0;
+    for (int64_t t = 0; t < N; ++t)
+        for (int k = 0; k < K; ++k) {
+            int32_t p = pos[t * K + k];
+            if (p < 0 || p >= cap) continue;
+            float wk = w[t * K + k];
+            for (int h = 0; h < H; ++h) {
+                float g = oracle_bf16_to_f32(grad_out[t * H + h]);
+                grad_rows[(int64_t)p * H + h] = oracle_f32_to_bf16(wk * g);
+            }
+        }
+}
+
+/* Combine backward, route-weight side: d out[t] / d w[t,k] = y[pos[t,k]], so
+ * the weight gradient is the dot product of that row with grad_out[t],
+ * computed here in double precision (the yardstick for the fp32 sum of the
+ * CUDA path). Entries with pos < 0 get 0. */
+void oracle_combine_backward_weights(const uint16_t* grad_out,
+                                     const uint16_t* y, const int32_t* pos,
+                                     int64_t N, int K, int H, int64_t cap,
+                                     double* grad_w) {
+    for (int64_t t = 0; t < N; ++t)
+        for (int k = 0; k < K; ++k) {
+            int32_t p = pos[t * K + k];
+            double acc = 0.0;
+            if (p >= 0 && p < cap)
+                for (int h = 0; h < H; ++h)
+                    acc += (double)oracle_bf16_to_f32(y[(int64_t)p * H + h]) *
+                           (double)oracle_bf16_to_f32(grad_out[t * H + h]);
+            grad_w[t * K + k] = acc;
+        }
+}
+
+/* gathered_route_weights: the per-row values of the receive side gathered
+ * back into token order, out[t,k] = row_vals[pos[t,k]] (0 where pos < 0). */
+void oracle_gather_row_values(const float* row_vals, const int32_t* pos,
+                              int64_t N, int K, int64_t cap, float* out) {
+    for (int64_t i = 0; i < N * K; ++i) {
+        int32_t p = pos[i];
+        out[i] = (p >= 0 && p < cap) ? row_vals[p] : 0.0f;
+    }
+}
