@@ -75,6 +75,17 @@ def bytes_prefetch(n_slots, H, I):
     return 3 * n_slots * H * I * 2 * 2
 
 
+def bytes_combine_backward(N, K, H, used_rows):
+    # grad_out and the K gathered expert-output rows read, every used
+    # receive row's gradient written (padding rows zeroed), grad_w written
+    return (N * H * 2 + N * K * H * 2 + N * K * 8 + used_rows * 4 +
+            used_rows * H * 2 + N * K * 4)
+
+
+def bytes_dispatch_backward(N, K, H):
+    return N * K * H * 2 + N * K * 4 + N * H * 2
+
+
 # --------------------------------------------------------------------------
 # environment helpers
 # --------------------------------------------------------------------------
@@ -247,6 +258,37 @@ class Path:
             self.W = [workloads.weight_buffer(rows, wl.H, wl.I, wl.seed + j,
                                               device=dev) for j in range(3)]
         self.launches_per_step = 4 + (2 if wl.B > 0 else 0)
+        self.backward = False
+
+    def enable_backward(self, seed_offset=0):
+        """Buffers of the backward pair: a synthetic gradient of the
+        combined output, gradients of the expert outputs / route weights /
+        token rows."""
+        wl, dev = self.wl, self.dev
+        self.backward = True
+        self.grad_out = workloads.bf16_normal((wl.N, wl.H), 4000 + wl.seed +
+                                              seed_offset, device=dev)
+        self.grad_rows = torch.empty(self.cap, wl.H, dtype=torch.bfloat16,
+                                     device=dev)
+        self.grad_w = torch.empty(wl.N, wl.K, dtype=torch.float32, device=dev)
+        self.grad_hidden = torch.empty(wl.N, wl.H, dtype=torch.bfloat16,
+                                       device=dev)
+        self.launches_per_step += 2
+
+    def combine_backward(self, io=None):
+        wl = self.wl
+        io = io or self.io()
+        self.ep.ep_combine_backward(self.grad_out, self.y, self.pos,
+                                    self.row_src, self.offsets, io["w"], wl.N,
+                                    wl.K, wl.E, wl.H, self.grad_rows,
+                                    self.grad_w, status=self.status,
+                                    cap=self.cap)
+
+    def dispatch_backward(self, io=None):
+        wl = self.wl
+        self.ep.ep_dispatch_backward(self.grad_rows, self.pos, wl.N, wl.K,
+                                     wl.H, self.grad_hidden,
+                                     status=self.status, cap=self.cap)
 
     def io(self):
         """The buffers a user hands in and gets back (one set)."""
@@ -287,6 +329,9 @@ class Path:
             self.plan_prefetch()
         self.dispatch(io)
         self.combine(io)
+        if self.backward:
+            self.combine_backward(io)
+            self.dispatch_backward(io)
 
 
 def run_gpu(args, wl):
@@ -308,6 +353,8 @@ def run_gpu(args, wl):
         return max_over_ranks(x, dev)
 
     path = Path(wl, dev, seed_offset=rank)
+    if args.backward:
+        path.enable_backward(seed_offset=rank)
     torch.cuda.synchronize()
     # warm-up (also settles the used-row count for byte accounting)
     for _ in range(args.warmup):
@@ -323,7 +370,9 @@ def run_gpu(args, wl):
     b_dis = bytes_dispatch(wl.N, wl.K, wl.H, wl.fp8, used)
     b_com = bytes_combine(wl.N, wl.K, wl.H)
     b_pre = bytes_prefetch(n_slots, wl.H, wl.I) if wl.B else 0
-    b_step = b_lay + b_dis + b_com + b_pre
+    b_cbw = bytes_combine_backward(wl.N, wl.K, wl.H, used) if args.backward else 0
+    b_dbw = bytes_dispatch_backward(wl.N, wl.K, wl.H) if args.backward else 0
+    b_step = b_lay + b_dis + b_com + b_pre + b_cbw + b_dbw
 
     # The K timed steps are captured once into a CUDA graph (the library is
     # capture-safe: no allocation, no synchronisation) and replayed once, so
@@ -368,7 +417,11 @@ def run_gpu(args, wl):
              "combine": path.combine}
     if wl.B > 0:
         parts["plan_prefetch"] = path.plan_prefetch
-    avg = {"plan_prefetch": 0.0}
+    if args.backward:
+        parts["combine_backward"] = path.combine_backward
+        parts["dispatch_backward"] = path.dispatch_backward
+    avg = {"plan_prefetch": 0.0, "combine_backward": 0.0,
+           "dispatch_backward": 0.0}
     for name, fn in parts.items():
         g = capture(fn, K)
         avg[name] = replay_ms(g) / K * 1e3     # us per launch
@@ -416,7 +469,9 @@ def run_gpu(args, wl):
                 "workload": wl.describe,
                 "step": ("ep_layout + " + ("ep_plan_balanced + "
                          "ep_prefetch_weights + " if wl.B else "") +
-                         "ep_dispatch + ep_combine"),
+                         "ep_dispatch + ep_combine" +
+                         (" + ep_combine_backward + ep_dispatch_backward"
+                          if args.backward else "")),
                 "bytes_per_step": b_step,
                 "used_rows": used,
                 "l2": "no flush: every step moves >4 GB, inputs larger "
@@ -438,6 +493,14 @@ def run_gpu(args, wl):
                 "dispatch_payload_GBps": round(
                     payload_dispatch(wl.N, wl.K, wl.H, wl.fp8) /
                     (avg["dispatch"] * 1e-6) / 1e9, 1),
+                "combine_backward_us": round(med["combine_backward"], 2),
+                "dispatch_backward_us": round(med["dispatch_backward"], 2),
+                "combine_backward_GBps": round(
+                    b_cbw / (avg["combine_backward"] * 1e-6) / 1e9, 1)
+                if args.backward else None,
+                "dispatch_backward_GBps": round(
+                    b_dbw / (avg["dispatch_backward"] * 1e-6) / 1e9, 1)
+                if args.backward else None,
                 "dispatch_bytes": b_dis, "combine_bytes": b_com,
                 "layout_bytes": b_lay, "prefetch_bytes": b_pre,
                 "frac_of_8TBps": {
@@ -640,6 +703,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="add the backward pair to the step")
     ap.add_argument("--cpu-sample-tokens", type=int, default=8192)
     ap.add_argument("--tokens-per-rank", type=int, default=None,
                     help="override S (smaller cases for profiling)")

@@ -6,8 +6,9 @@ from ._binding import (  # noqa: F401
     EP_DEV_BAD_EXPERT, EP_DEV_CAPACITY, EP_DEV_PLAN_TOTAL, EP_DEV_SLOTS,
     EP_DEV_TIMEOUT, EP_ERR_ALIGNMENT, EP_ERR_CAPACITY, EP_ERR_CUDA,
     EP_ERR_INVALID_ARG, EP_ERR_WORKSPACE, EP_OK, EPError, ep_abi_version,
-    ep_capacity_bound, ep_combine, ep_debug_bounded_wait,
-    ep_debug_e4m3_encode, ep_debug_quantize, ep_dispatch, ep_layout, ep_layout_workspace_bytes,
+    ep_capacity_bound, ep_combine, ep_combine_backward, ep_debug_bounded_wait,
+    ep_debug_e4m3_encode, ep_debug_quantize, ep_dispatch,
+    ep_dispatch_backward, ep_gather_route_weights, ep_layout, ep_layout_workspace_bytes,
     ep_plan_balanced, ep_prefetch_weights, ep_strerror, lib, library_path,
     strerror)
 from .buffer import EPBuffer  # noqa: F401

@@ -83,6 +83,13 @@ def _declare(L):
                               P, P, i32, P, P]
     L.ep_combine.restype = i32
     L.ep_combine.argtypes = [P, P, P, i64, i32, i32, i64, P, i32, P, P]
+    L.ep_dispatch_backward.restype = i32
+    L.ep_dispatch_backward.argtypes = [P, P, i64, i32, i32, i64, P, i32, P, P]
+    L.ep_combine_backward.restype = i32
+    L.ep_combine_backward.argtypes = [P, P, P, P, P, P, i64, i32, i32, i32,
+                                      i64, P, P, i32, P, P]
+    L.ep_gather_route_weights.restype = i32
+    L.ep_gather_route_weights.argtypes = [P, P, i64, i32, i64, P, P]
     L.ep_plan_balanced.restype = i32
     L.ep_plan_balanced.argtypes = [P, i32, i32, i32, i32, i32, P, P, P, P, P,
                                    P, P]
@@ -221,6 +228,51 @@ def ep_combine(expert_out, pos, route_weights, num_tokens, K, H, out,
         _ptr(status, "status", _I32, 1, optional=True),
         _stream(stream))
     _check(rc, "ep_combine")
+
+
+def ep_dispatch_backward(grad_recv, pos, num_tokens, K, H, grad_hidden,
+                         num_sms=0, status=None, cap=None, stream=None):
+    """grad_hidden[t] = bf16(sum_k grad_recv[pos[t,k]]) in fp32, k order."""
+    cap = grad_recv.shape[0] if cap is None else int(cap)
+    rc = lib().ep_dispatch_backward(
+        _ptr(grad_recv, "grad_recv", _BF16, cap * H),
+        _ptr(pos, "pos", _I32, num_tokens * K), num_tokens, K, H, cap,
+        _ptr(grad_hidden, "grad_hidden", _BF16, num_tokens * H),
+        int(num_sms), _ptr(status, "status", _I32, 1, optional=True),
+        _stream(stream))
+    _check(rc, "ep_dispatch_backward")
+
+
+def ep_combine_backward(grad_out, expert_out, pos, row_src, expert_offsets,
+                        route_weights, num_tokens, K, E, H, grad_expert_out,
+                        grad_route_weights, num_sms=0, status=None, cap=None,
+                        stream=None):
+    """Gradients of combine: scaled rows and per-entry dot products."""
+    cap = expert_out.shape[0] if cap is None else int(cap)
+    rc = lib().ep_combine_backward(
+        _ptr(grad_out, "grad_out", _BF16, num_tokens * H),
+        _ptr(expert_out, "expert_out", _BF16, cap * H),
+        _ptr(pos, "pos", _I32, num_tokens * K),
+        _ptr(row_src, "row_src", _I32, cap),
+        _ptr(expert_offsets, "expert_offsets", _I32, E + 1),
+        _ptr(route_weights, "route_weights", _F32, num_tokens * K),
+        num_tokens, K, E, H, cap,
+        _ptr(grad_expert_out, "grad_expert_out", _BF16, cap * H),
+        _ptr(grad_route_weights, "grad_route_weights", _F32, num_tokens * K),
+        int(num_sms), _ptr(status, "status", _I32, 1, optional=True),
+        _stream(stream))
+    _check(rc, "ep_combine_backward")
+
+
+def ep_gather_route_weights(row_values, pos, num_tokens, K, out, cap=None,
+                            stream=None):
+    """out[t,k] = row_values[pos[t,k]] (gathered_route_weights)."""
+    cap = row_values.numel() if cap is None else int(cap)
+    rc = lib().ep_gather_route_weights(
+        _ptr(row_values, "row_values", _F32, cap),
+        _ptr(pos, "pos", _I32, num_tokens * K), num_tokens, K, cap,
+        _ptr(out, "out", _F32, num_tokens * K), _stream(stream))
+    _check(rc, "ep_gather_route_weights")
 
 
 def ep_plan_balanced(tokens_per_expert, R, S, K, E, B, plan_cu, plan_expert,

@@ -8,7 +8,7 @@
 
 namespace {
 
-constexpr int kAbiVersion = 1;
+constexpr int kAbiVersion = 2;
 constexpr int kMaxK = 32;
 constexpr int kMaxH = 32768;
 constexpr int64_t kMaxEntries = (int64_t(1) << 30) - 1;
@@ -148,6 +148,62 @@ int ep_combine(const void* expert_out, const int32_t* pos,
   return cuda_rc(ep::launch_combine(expert_out, pos, route_weights, num_tokens,
                                     K, H, cap, out, sms_or_all(num_sms),
                                     status, as_stream(stream)));
+}
+
+int ep_dispatch_backward(const void* grad_recv, const int32_t* pos,
+                         int64_t num_tokens, int K, int H, int64_t cap,
+                         void* grad_hidden, int num_sms, int32_t* status,
+                         void* stream) {
+  if (num_tokens < 0 || K < 1 || K > kMaxK || H < 8 || H > kMaxH ||
+      H % 8 != 0 || cap < 0 || cap > INT32_MAX || num_sms < 0 ||
+      num_tokens * K > kMaxEntries)
+    return EP_ERR_INVALID_ARG;
+  if (!status_ok(status)) return EP_ERR_ALIGNMENT;
+  if (num_tokens == 0) return EP_OK;
+  if (!aligned16(pos) || !aligned16(grad_hidden)) return EP_ERR_ALIGNMENT;
+  if (cap > 0 && !aligned16(grad_recv)) return EP_ERR_ALIGNMENT;
+  return cuda_rc(ep::launch_combine(grad_recv, pos, nullptr, num_tokens, K, H,
+                                    cap, grad_hidden, sms_or_all(num_sms),
+                                    status, as_stream(stream)));
+}
+
+int ep_combine_backward(const void* grad_out, const void* expert_out,
+                        const int32_t* pos, const int32_t* row_src,
+                        const int32_t* expert_offsets,
+                        const float* route_weights, int64_t num_tokens, int K,
+                        int E, int H, int64_t cap, void* grad_expert_out,
+                        float* grad_route_weights, int num_sms,
+                        int32_t* status, void* stream) {
+  if (num_tokens < 0 || K < 1 || K > kMaxK || E < 1 || H < 8 || H > kMaxH ||
+      H % 8 != 0 || cap < 0 || cap > INT32_MAX || num_sms < 0 ||
+      num_tokens * K > kMaxEntries)
+    return EP_ERR_INVALID_ARG;
+  if (!aligned16(expert_offsets) || !status_ok(status)) return EP_ERR_ALIGNMENT;
+  if (num_tokens > 0 && (!aligned16(grad_out) || !aligned16(pos) ||
+                         !aligned16(route_weights) ||
+                         !aligned16(grad_route_weights)))
+    return EP_ERR_ALIGNMENT;
+  if (cap > 0 && (!aligned16(expert_out) || !aligned16(row_src) ||
+                  !aligned16(grad_expert_out)))
+    return EP_ERR_ALIGNMENT;
+  if (num_tokens == 0 && cap == 0) return EP_OK;
+  return cuda_rc(ep::launch_combine_backward(
+      grad_out, expert_out, pos, row_src, expert_offsets, route_weights,
+      num_tokens, K, E, H, cap, grad_expert_out, grad_route_weights,
+      sms_or_all(num_sms), status, as_stream(stream)));
+}
+
+int ep_gather_route_weights(const float* row_values, const int32_t* pos,
+                            int64_t num_tokens, int K, int64_t cap, float* out,
+                            void* stream) {
+  if (num_tokens < 0 || K < 1 || K > kMaxK || cap < 0 || cap > INT32_MAX ||
+      num_tokens * K > kMaxEntries)
+    return EP_ERR_INVALID_ARG;
+  if (num_tokens == 0) return EP_OK;
+  if (!aligned16(pos) || !aligned16(out)) return EP_ERR_ALIGNMENT;
+  if (cap > 0 && !aligned16(row_values)) return EP_ERR_ALIGNMENT;
+  return cuda_rc(ep::launch_gather_row_values(row_values, pos, num_tokens * K,
+                                              cap, out, as_stream(stream)));
 }
 
 int ep_plan_balanced(const int32_t* tokens_per_expert, int R, int S, int K,

@@ -57,14 +57,14 @@ __global__ void __launch_bounds__(kCombineMaxThreads)
   const int V = H >> 3;
   for (int64_t t = blockIdx.x; t < N; t += gridDim.x) {
     const int32_t* pt = pos + t * K;
-    const float* wt = w + t * K;
+    const float* wt = w ? w + t * K : nullptr;  // NULL: unit weights
     if constexpr (KT > 0) {
       int64_t rowoff[KT];
       float wk[KT];
 #pragma unroll
       for (int k = 0; k < KT; ++k) {
         const int32_t p = __ldg(pt + k);
-        wk[k] = __ldg(wt + k);
+        wk[k] = w ? __ldg(wt + k) : 1.0f;
         const bool ok = p >= 0 && p < cap;
         if (p >= cap && threadIdx.x == 0) report(status, EP_DEV_CAPACITY);
         rowoff[k] = ok ? int64_t(p) * H : int64_t(-1);
@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(kCombineMaxThreads)
             wk[j] = 0.f;
             if (k0 + j < K) {
               const int32_t p = __ldg(pt + k0 + j);
-              wk[j] = __ldg(wt + k0 + j);
+              wk[j] = w ? __ldg(wt + k0 + j) : 1.0f;
               if (p >= 0 && p < cap) off[j] = int64_t(p) * H;
               if (p >= cap && v == threadIdx.x && threadIdx.x == 0)
                 report(status, EP_DEV_CAPACITY);
@@ -189,7 +189,7 @@ __global__ void __launch_bounds__((kTmaMaxConsumerWarps + 1) * 32, 1)
     if (u < units && lane < K) {
       const int64_t t0 = u / sh.parts;
       p_n = __ldg(pos + t0 * K + lane);
-      w_n = __ldg(w + t0 * K + lane);
+      w_n = w ? __ldg(w + t0 * K + lane) : 1.0f;
     }
     for (; u < units; u += gridDim.x, ++it) {
       const int64_t t = u / sh.parts;
@@ -204,7 +204,7 @@ __global__ void __launch_bounds__((kTmaMaxConsumerWarps + 1) * 32, 1)
         if (un < units && lane < K) {
           const int64_t tn = un / sh.parts;
           p_n = __ldg(pos + tn * K + lane);
-          w_n = __ldg(w + tn * K + lane);
+          w_n = w ? __ldg(w + tn * K + lane) : 1.0f;
         }
       }
       const bool valid = lane < K && p >= 0 && p < cap;

@@ -33,9 +33,24 @@ cudaError_t launch_dispatch(const void* hidden, const float* w,
                             float* recv_scales, float* recv_w, int num_sms,
                             int32_t* status, cudaStream_t stream);
 
+// w == NULL: unit weights (dispatch backward)
 cudaError_t launch_combine(const void* y, const int32_t* pos, const float* w,
                            int64_t N, int K, int H, int64_t cap, void* out,
                            int num_sms, int32_t* status, cudaStream_t stream);
+
+// ---- backward pair ---------------------------------------------------------
+
+cudaError_t launch_combine_backward(const void* grad_out, const void* y,
+                                    const int32_t* pos, const int32_t* row_src,
+                                    const int32_t* expert_offsets,
+                                    const float* w, int64_t N, int K, int E,
+                                    int H, int64_t cap, void* grad_rows,
+                                    float* grad_w, int num_sms,
+                                    int32_t* status, cudaStream_t stream);
+
+cudaError_t launch_gather_row_values(const float* vals, const int32_t* pos,
+                                     int64_t n, int64_t cap, float* out,
+                                     cudaStream_t stream);
 
 // ---- balanced plan / prefetch ---------------------------------------------
 

@@ -199,6 +199,69 @@ EP_API int ep_combine(const void* expert_out, const int32_t* pos,
                void* stream);
 
 /*
+ * ep_dispatch_backward -- gradient of the bf16 dispatch with respect to the
+ * token rows: each token's gradient is the sum of the gradients of its K
+ * receive rows, grad_hidden[t,h] = bf16_rne(acc), acc = +0 then for
+ * k = 0..K-1 acc += float(grad_recv[pos[t,k], h]) in fp32 (combine with
+ * unit weights). ("DeepSeek开源周第二天：DeepEP深度分析", "DeepEP介绍":
+ * kernels for training as well as inference.)
+ *
+ * in   grad_recv         bf16 [cap, H]: gradient of the receive buffer
+ *      pos               int32 [N, K] from ep_layout (entries < 0 skipped)
+ * out  grad_hidden       bf16 [N, H]
+ *      status            EP_DEV_CAPACITY may be OR-ed in
+ */
+EP_API int ep_dispatch_backward(const void* grad_recv, const int32_t* pos,
+                                int64_t num_tokens, int K, int H, int64_t cap,
+                                void* grad_hidden, int num_sms,
+                                int32_t* status, void* stream);
+
+/*
+ * ep_combine_backward -- gradients of the combine with respect to the expert
+ * outputs and to the route weights ("DeepSeek开源周第二天：DeepEP深度分析",
+ * "DeepEP介绍": training kernels; "MoonEP核心功能深度剖析", "快速上手":
+ * combine's outputs include what the backward pass needs).
+ *
+ * in   grad_out          bf16 [N, H]: gradient of the combined output
+ *      expert_out        bf16 [cap, H]: the forward pass's expert outputs y
+ *      pos, row_src,
+ *      expert_offsets    from ep_layout
+ *      route_weights     fp32 [N, K]
+ * out  grad_expert_out   bf16 [cap, H]: row pos[t,k] <- bf16_rne(w[t,k] *
+ *                        float(grad_out[t])) (fp32 product); padding rows
+ *                        (row_src == -1 below off[E]) <- 0; rows >= off[E]
+ *                        untouched
+ *      grad_route_weights fp32 [N, K]: sum over h of float(y[pos[t,k], h]) *
+ *                        float(grad_out[t, h]) in fp32; the summation order
+ *                        is fixed by the implementation (deterministic), so
+ *                        it matches the exact sum within the fp32 rounding
+ *                        bound H * 2^-24 * sum|terms|; 0 where pos < 0
+ *      status            EP_DEV_CAPACITY may be OR-ed in
+ */
+EP_API int ep_combine_backward(const void* grad_out, const void* expert_out,
+                               const int32_t* pos, const int32_t* row_src,
+                               const int32_t* expert_offsets,
+                               const float* route_weights, int64_t num_tokens,
+                               int K, int E, int H, int64_t cap,
+                               void* grad_expert_out,
+                               float* grad_route_weights, int num_sms,
+                               int32_t* status, void* stream);
+
+/*
+ * ep_gather_route_weights -- per-row values of the receive side gathered
+ * back into token order, out[t,k] = row_values[pos[t,k]] (0 where pos < 0):
+ * the pages' gathered_route_weights_sk ("MoonEP核心功能深度剖析", "快速上手":
+ * combine(...) -> output_sh, gathered_route_weights_sk).
+ *
+ * in   row_values        fp32 [cap] (e.g. recv_weights from ep_dispatch)
+ *      pos               int32 [N, K]
+ * out  out               fp32 [N, K]
+ */
+EP_API int ep_gather_route_weights(const float* row_values, const int32_t* pos,
+                                   int64_t num_tokens, int K, int64_t cap,
+                                   float* out, void* stream);
+
+/*
  * ep_plan_balanced -- the perfectly balanced plan ("MoonEP核心功能深度剖析",
  * "1. 完美负载平衡": every rank receives exactly S*K rows however skewed the
  * routing, through a few redundant experts planned online; "3. 智能内存管理":

@@ -41,7 +41,7 @@ def test_library_is_the_in_tree_build():
 
 
 def test_pure_host_entry_points():
-    assert ep.ep_abi_version() == 1
+    assert ep.ep_abi_version() == 2
     assert ep.ep_capacity_bound(32768, 8, 256, 128) == 32768 * 8 + 256 * 127
     assert ep.ep_capacity_bound(10, 2, 4, 1) == 20
     assert ep.ep_capacity_bound(-1, 2, 4, 1) < 0
