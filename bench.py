@@ -86,6 +86,14 @@ def bytes_dispatch_backward(N, K, H):
     return N * K * H * 2 + N * K * 4 + N * H * 2
 
 
+def bytes_reduce_slot_grads(slots, H, I):
+    """fp32 gradients: per expert with n slots, its row read and written and
+    its n slot rows read, for three projections."""
+    import collections
+    groups = collections.Counter(int(e) for e in slots.ravel() if e >= 0)
+    return 3 * sum(n + 2 for n in groups.values()) * H * I * 4
+
+
 # --------------------------------------------------------------------------
 # environment helpers
 # --------------------------------------------------------------------------
@@ -274,6 +282,16 @@ class Path:
         self.grad_hidden = torch.empty(wl.N, wl.H, dtype=torch.bfloat16,
                                        device=dev)
         self.launches_per_step += 2
+        if wl.B > 0:
+            rows = wl.E + wl.R * wl.B
+            self.GW = [torch.zeros(rows, wl.H, wl.I, dtype=torch.float32,
+                                   device=dev) for _ in range(3)]
+            self.launches_per_step += 1
+
+    def reduce_slot_grads(self, io=None):
+        wl = self.wl
+        self.ep.ep_reduce_slot_grads(self.plan["slot"], wl.R, wl.E, wl.B,
+                                     *self.GW)
 
     def combine_backward(self, io=None):
         wl = self.wl
@@ -332,6 +350,8 @@ class Path:
         if self.backward:
             self.combine_backward(io)
             self.dispatch_backward(io)
+            if self.wl.B > 0:
+                self.reduce_slot_grads(io)
 
 
 def run_gpu(args, wl):
@@ -372,7 +392,9 @@ def run_gpu(args, wl):
     b_pre = bytes_prefetch(n_slots, wl.H, wl.I) if wl.B else 0
     b_cbw = bytes_combine_backward(wl.N, wl.K, wl.H, used) if args.backward else 0
     b_dbw = bytes_dispatch_backward(wl.N, wl.K, wl.H) if args.backward else 0
-    b_step = b_lay + b_dis + b_com + b_pre + b_cbw + b_dbw
+    b_red = (bytes_reduce_slot_grads(path.plan["slot"].cpu().numpy(), wl.H,
+                                     wl.I) if args.backward and wl.B else 0)
+    b_step = b_lay + b_dis + b_com + b_pre + b_cbw + b_dbw + b_red
 
     # The K timed steps are captured once into a CUDA graph (the library is
     # capture-safe: no allocation, no synchronisation) and replayed once, so
@@ -420,8 +442,10 @@ def run_gpu(args, wl):
     if args.backward:
         parts["combine_backward"] = path.combine_backward
         parts["dispatch_backward"] = path.dispatch_backward
+        if wl.B > 0:
+            parts["reduce_slot_grads"] = path.reduce_slot_grads
     avg = {"plan_prefetch": 0.0, "combine_backward": 0.0,
-           "dispatch_backward": 0.0}
+           "dispatch_backward": 0.0, "reduce_slot_grads": 0.0}
     for name, fn in parts.items():
         g = capture(fn, K)
         avg[name] = replay_ms(g) / K * 1e3     # us per launch
@@ -471,7 +495,9 @@ def run_gpu(args, wl):
                          "ep_prefetch_weights + " if wl.B else "") +
                          "ep_dispatch + ep_combine" +
                          (" + ep_combine_backward + ep_dispatch_backward"
-                          if args.backward else "")),
+                          if args.backward else "") +
+                         (" + ep_reduce_slot_grads"
+                          if args.backward and wl.B else "")),
                 "bytes_per_step": b_step,
                 "used_rows": used,
                 "l2": "no flush: every step moves >4 GB, inputs larger "
@@ -501,6 +527,10 @@ def run_gpu(args, wl):
                 "dispatch_backward_GBps": round(
                     b_dbw / (avg["dispatch_backward"] * 1e-6) / 1e9, 1)
                 if args.backward else None,
+                "reduce_slot_grads_us": round(med["reduce_slot_grads"], 2),
+                "reduce_slot_grads_GBps": round(
+                    b_red / (avg["reduce_slot_grads"] * 1e-6) / 1e9, 1)
+                if b_red else None,
                 "dispatch_bytes": b_dis, "combine_bytes": b_com,
                 "layout_bytes": b_lay, "prefetch_bytes": b_pre,
                 "frac_of_8TBps": {

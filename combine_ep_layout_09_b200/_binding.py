@@ -95,6 +95,8 @@ def _declare(L):
                                    P, P]
     L.ep_prefetch_weights.restype = i32
     L.ep_prefetch_weights.argtypes = [P, i32, i32, i32, i64, P, P, P, i32, P]
+    L.ep_reduce_slot_grads.restype = i32
+    L.ep_reduce_slot_grads.argtypes = [P, i32, i32, i32, i64, P, P, P, i32, P]
     L.ep_debug_e4m3_encode.restype = i32
     L.ep_debug_e4m3_encode.argtypes = [P, P, i64, P]
     L.ep_debug_quantize.restype = i32
@@ -307,6 +309,23 @@ def ep_prefetch_weights(slot_expert, R, E, B, gate, up, down, num_sms=0,
         _ptr(down, "down", _W16),
         int(num_sms), _stream(stream))
     _check(rc, "ep_prefetch_weights")
+
+
+def ep_reduce_slot_grads(slot_expert, R, E, B, grad_gate, grad_up,
+                         grad_down, num_sms=0, stream=None):
+    """Add every prefetched copy's gradient into its expert's row."""
+    rows = E + R * B
+    elems = grad_gate[0].numel() if grad_gate.shape[0] > 0 else 0
+    for name, t in (("grad_gate", grad_gate), ("grad_up", grad_up),
+                    ("grad_down", grad_down)):
+        if t.shape[0] != rows or t[0].numel() != elems:
+            raise ValueError(f"{name} must be [E + R*B, ...] like grad_gate")
+    rc = lib().ep_reduce_slot_grads(
+        _ptr(slot_expert, "slot_expert", _I32, R * B, optional=(B == 0)),
+        R, E, B, elems,
+        _ptr(grad_gate, "grad_gate", _F32), _ptr(grad_up, "grad_up", _F32),
+        _ptr(grad_down, "grad_down", _F32), int(num_sms), _stream(stream))
+    _check(rc, "ep_reduce_slot_grads")
 
 
 def ep_debug_e4m3_encode(x, out, stream=None):

@@ -239,6 +239,24 @@ int ep_prefetch_weights(const int32_t* slot_expert, int R, int E, int B,
                                      as_stream(stream)));
 }
 
+int ep_reduce_slot_grads(const int32_t* slot_expert, int R, int E, int B,
+                         int64_t elems_per_expert, float* grad_gate,
+                         float* grad_up, float* grad_down, int num_sms,
+                         void* stream) {
+  if (R < 1 || E < 1 || B < 0 || elems_per_expert < 0 ||
+      elems_per_expert % 4 != 0 || num_sms < 0 || int64_t(R) * B > 1024)
+    return EP_ERR_INVALID_ARG;
+  if (B == 0 || elems_per_expert == 0) return EP_OK;
+  if (!aligned16(slot_expert) || !aligned16(grad_gate) || !aligned16(grad_up) ||
+      !aligned16(grad_down))
+    return EP_ERR_ALIGNMENT;
+  return cuda_rc(ep::launch_reduce_slot_grads(slot_expert, R, E, B,
+                                              elems_per_expert, grad_gate,
+                                              grad_up, grad_down,
+                                              sms_or_all(num_sms),
+                                              as_stream(stream)));
+}
+
 int ep_debug_e4m3_encode(const float* x, uint8_t* out, int64_t n,
                          void* stream) {
   if (n < 0) return EP_ERR_INVALID_ARG;

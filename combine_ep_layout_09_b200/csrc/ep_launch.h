@@ -64,6 +64,11 @@ cudaError_t launch_prefetch(const int32_t* slot_expert, int R, int E, int B,
                             int64_t elems, void* gate, void* up, void* down,
                             int num_sms, cudaStream_t stream);
 
+cudaError_t launch_reduce_slot_grads(const int32_t* slot_expert, int R, int E,
+                                     int B, int64_t elems, float* g0, float* g1,
+                                     float* g2, int num_sms,
+                                     cudaStream_t stream);
+
 // ---- diagnostics ----------------------------------------------------------
 
 cudaError_t launch_debug_e4m3(const float* x, uint8_t* out, int64_t n,

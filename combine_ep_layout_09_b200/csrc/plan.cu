@@ -264,6 +264,77 @@ __global__ void __launch_bounds__(32)
   bulk_wait_all<0>();
 }
 
+// Slot-gradient reduce ("MoonEP核心功能深度剖析", "3. 智能内存管理", 图4: the
+// gradient buffer mirrors the weight buffer and the prefetched copies'
+// gradients are reduced into the owners' rows). Each CTA compacts the used
+// slots in (d, b) order; the first slot of each expert heads its group.
+// Units are (group, projection, chunk of float4 vectors): the expert's row
+// plus its slots' rows, added in (d, b) order in fp32, as the definition
+// states; slot rows are left as they are.
+constexpr int kRedThreads = 256;
+constexpr int64_t kRedVec = 4096;  // float4 vectors per unit (64 KB)
+
+__global__ void __launch_bounds__(kRedThreads)
+    k_reduce_slot_grads(const int32_t* __restrict__ slot_expert, int RB, int E,
+                        int64_t vecs, float4* __restrict__ g0,
+                        float4* __restrict__ g1, float4* __restrict__ g2) {
+  __shared__ int s_slot[kMaxSlotList], s_exp[kMaxSlotList], s_head[kMaxSlotList];
+  __shared__ int s_n, s_nh;
+  const int tid = threadIdx.x, lane = tid & 31;
+  if (tid < 32) {
+    int n = 0;
+    for (int b = 0; b < RB; b += 32) {
+      const int slot = b + lane;
+      const int32_t e = slot < RB ? __ldg(slot_expert + slot) : -1;
+      const bool used = e >= 0 && e < E;
+      const unsigned m = __ballot_sync(0xffffffffu, used);
+      if (used) {
+        const int at = n + __popc(m & ((1u << lane) - 1u));
+        s_slot[at] = slot;
+        s_exp[at] = e;
+      }
+      n += __popc(m);
+    }
+    if (lane == 0) s_n = n;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int nh = 0;
+    for (int j = 0; j < s_n; ++j) {
+      bool first = true;
+      for (int jj = 0; jj < j && first; ++jj) first = s_exp[jj] != s_exp[j];
+      if (first) s_head[nh++] = j;
+    }
+    s_nh = nh;
+  }
+  __syncthreads();
+  const int n = s_n;
+  const int64_t nchunk = (vecs + kRedVec - 1) / kRedVec;
+  const int64_t units = int64_t(s_nh) * 3 * nchunk;
+  for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
+    const int64_t f = u / (3 * nchunk);
+    const int64_t rem = u - f * 3 * nchunk;
+    const int proj = int(rem / nchunk);
+    const int64_t ch = rem - int64_t(proj) * nchunk;
+    const int j0 = s_head[f];
+    const int e = s_exp[j0];
+    float4* G = proj == 0 ? g0 : (proj == 1 ? g1 : g2);
+    const int64_t lo = ch * kRedVec, hi = min(vecs, lo + kRedVec);
+    for (int64_t v = lo + tid; v < hi; v += kRedThreads) {
+      float4 acc = G[int64_t(e) * vecs + v];
+      for (int j = j0; j < n; ++j) {
+        if (s_exp[j] != e) continue;
+        const float4 x = G[(int64_t(E) + s_slot[j]) * vecs + v];
+        acc.x = acc.x + x.x;
+        acc.y = acc.y + x.y;
+        acc.z = acc.z + x.z;
+        acc.w = acc.w + x.w;
+      }
+      G[int64_t(e) * vecs + v] = acc;
+    }
+  }
+}
+
 __global__ void k_debug_e4m3(const float* __restrict__ x, uint8_t* __restrict__ out,
                              int64_t n) {
   const int64_t pairs = (n + 1) / 2;
@@ -340,6 +411,22 @@ cudaError_t launch_prefetch(const int32_t* slot_expert, int R, int E, int B,
   k_prefetch<<<int(grid), kCopyThreads, 0, stream>>>(
       slot_expert, int(RB), E, vecs, static_cast<uint4*>(gate),
       static_cast<uint4*>(up), static_cast<uint4*>(down));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reduce_slot_grads(const int32_t* slot_expert, int R, int E,
+                                     int B, int64_t elems, float* g0, float* g1,
+                                     float* g2, int num_sms,
+                                     cudaStream_t stream) {
+  const int64_t RB = int64_t(R) * B;
+  if (RB == 0 || elems == 0) return cudaSuccess;
+  const int64_t vecs = elems / 4;
+  const int64_t nchunk = (vecs + kRedVec - 1) / kRedVec;
+  const int64_t grid = std::max<int64_t>(
+      1, std::min<int64_t>(RB * 3 * nchunk, int64_t(num_sms) * 4));
+  k_reduce_slot_grads<<<int(grid), kRedThreads, 0, stream>>>(
+      slot_expert, int(RB), E, vecs, reinterpret_cast<float4*>(g0),
+      reinterpret_cast<float4*>(g1), reinterpret_cast<float4*>(g2));
   return cudaGetLastError();
 }
 

@@ -312,6 +312,27 @@ EP_API int ep_prefetch_weights(const int32_t* slot_expert, int R, int E, int B,
                         int64_t elems_per_expert, void* gate, void* up,
                         void* down, int num_sms, void* stream);
 
+/*
+ * ep_reduce_slot_grads -- fold the gradients of the prefetched expert copies
+ * back into the experts' own gradient rows ("MoonEP核心功能深度剖析",
+ * "3. 智能内存管理", 图4: the gradient buffer mirrors the weight buffer, rows
+ * [0, E) the owners' gradients, the slots' gradients reduced into them).
+ *
+ * in   slot_expert       int32 [R, B] from ep_plan_balanced; R*B <= 1024
+ *      elems_per_expert  fp32 elements per expert row of one projection
+ *                        (H*I), a multiple of 4
+ * in/out grad_gate, grad_up, grad_down  fp32 [E + R*B, elems_per_expert]:
+ *                        row e += row E + d*B + b for every slot with
+ *                        slot_expert[d,b] == e, the slots added in (d, b)
+ *                        order with one fp32 addition each; slot rows and
+ *                        rows of experts without slots are left as they are
+ *      num_sms           SMs to use, 0 = all
+ */
+EP_API int ep_reduce_slot_grads(const int32_t* slot_expert, int R, int E,
+                                int B, int64_t elems_per_expert,
+                                float* grad_gate, float* grad_up,
+                                float* grad_down, int num_sms, void* stream);
+
 /* ---- diagnostics (used by the test-suite) ------------------------------ */
 
 /* out[i] = e4m3 code of x[i] through the same device conversion the FP8

@@ -20,6 +20,8 @@ Parity status of each function (what pins it, in tests/test_oracle_*.py):
   plan_balanced                           brute-force row-by-row planner,
                                           every rank exactly S*K rows
   prefetch                                slot rows equal source rows
+  reduce_slot_grads                       brute force, exact on integer
+                                          gradients, sum preserved (fp64)
   dispatch_backward                       adjoint of bf16 dispatch (fp64
                                           inner products), brute force
   combine_backward_rows / _weights        adjoint of combine, finite
@@ -94,6 +96,8 @@ def lib():
                                                       i64, P]
         L.oracle_gather_row_values.restype = None
         L.oracle_gather_row_values.argtypes = [P, P, i64, i32, i64, P]
+        L.oracle_reduce_slot_grads.restype = None
+        L.oracle_reduce_slot_grads.argtypes = [P, i32, i32, i32, i64, P]
         L.oracle_plan_balanced.restype = i32
         L.oracle_plan_balanced.argtypes = [P, i32, i32, i32, i32, i32, P, P,
                                            P, P, P]
@@ -323,6 +327,18 @@ def plan_balanced(counts: np.ndarray, R: int, S: int, K: int, B: int):
                                     _p(wr), _p(nseg), _p(slots))
     return dict(cu=cu, expert=ex, wrow=wr, nseg=nseg, slot_expert=slots,
                 status=st)
+
+
+def reduce_slot_grads(slot_expert: np.ndarray, E: int,
+                      G: np.ndarray) -> np.ndarray:
+    """-> a copy of the fp32 gradient buffer G [E+R*B, ...] with every used
+    slot's gradient added into its expert's row, in (d, b) order."""
+    slot_expert = _c(slot_expert, np.int32)
+    R, B = slot_expert.shape
+    G = np.array(G, dtype=np.float32, order="C", copy=True)
+    elems = int(np.prod(G.shape[1:]))
+    lib().oracle_reduce_slot_grads(_p(slot_expert), R, E, B, elems, _p(G))
+    return G
 
 
 def prefetch(slot_expert: np.ndarray, E: int, W: np.ndarray) -> np.ndarray:

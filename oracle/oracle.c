@@ -500,3 +500,22 @@ void oracle_gather_row_values(const float* row_vals, const int32_t* pos,
         out[i] = (p >= 0 && p < cap) ? row_vals[p] : 0.0f;
     }
 }
+
+/* Redundant-slot gradient reduce [MEP "3. 智能内存管理", 图4: the gradient
+ * buffer mirrors the weight buffer; gradients of the prefetched copies are
+ * reduced into the owners' rows]. G is one projection's gradient buffer
+ * [E + R*B, elems] in fp32: rows [0, E) hold each expert's gradient, row
+ * E + d*B + b the gradient that rank d computed for its copy of expert
+ * slot_expert[d*B+b]. Every used slot is added into its expert's row, slots
+ * in (d, b) order, one fp32 addition each; slot rows are left as they are. */
+void oracle_reduce_slot_grads(const int32_t* slot_expert, int R, int E, int B,
+                              int64_t elems, float* G) {
+    for (int d = 0; d < R; ++d)
+        for (int b = 0; b < B; ++b) {
+            int32_t e = slot_expert[d * B + b];
+            if (e < 0 || e >= E) continue;
+            int64_t src = (int64_t)E + (int64_t)d * B + b;
+            for (int64_t i = 0; i < elems; ++i)
+                G[(int64_t)e * elems + i] = G[(int64_t)e * elems + i] + G[src * elems + i];
+        }
+}

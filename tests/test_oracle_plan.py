@@ -156,3 +156,39 @@ def test_prefetch_copies_slots_only():
     np.testing.assert_array_equal(out, ref)
     assert np.array_equal(out[:E], W[:E])
     assert np.array_equal(out[E + 2], W[E + 2])     # unused slots untouched
+
+
+def test_reduce_slot_grads_exact_on_integers():
+    # integer-valued fp32 gradients: every sum is exact, so the result is
+    # the brute-force sum whatever the order
+    R, B, E = 4, 2, 6
+    rng = np.random.default_rng(8)
+    G = rng.integers(-1000, 1000, size=(E + R * B, 3, 5)).astype(np.float32)
+    slots = np.array([[2, -1], [2, 5], [-1, -1], [0, 2]], np.int32)
+    out = oracle.reduce_slot_grads(slots, E, G)
+    ref = G.copy()
+    for d in range(R):
+        for b in range(B):
+            if slots[d, b] >= 0:
+                ref[slots[d, b]] += G[E + d * B + b]
+    np.testing.assert_array_equal(out, ref)
+    np.testing.assert_array_equal(out[E:], G[E:])        # slot rows kept
+    assert np.array_equal(out[1], G[1]) and np.array_equal(out[3], G[3])
+
+
+def test_reduce_slot_grads_preserves_the_total_and_order():
+    R, B, E = 3, 2, 4
+    rng = np.random.default_rng(9)
+    G = rng.standard_normal((E + R * B, 64)).astype(np.float32)
+    slots = np.array([[1, 3], [1, -1], [0, 1]], np.int32)
+    out = oracle.reduce_slot_grads(slots, E, G)
+    used = [(d, b) for d in range(R) for b in range(B) if slots[d, b] >= 0]
+    total_before = G[:E].astype(np.float64).sum(0) + sum(
+        G[E + d * B + b].astype(np.float64) for d, b in used)
+    total_after = out[:E].astype(np.float64).sum(0)
+    np.testing.assert_allclose(total_after, total_before, rtol=0, atol=1e-5)
+    # expert 1 gets slots (0,0), (1,0), (2,1) added left to right in fp32
+    acc = G[1].copy()
+    for d, b in [(0, 0), (1, 0), (2, 1)]:
+        acc = (acc + G[E + d * B + b]).astype(np.float32)
+    np.testing.assert_array_equal(out[1], acc)

@@ -143,3 +143,51 @@ def test_prefetch_forms_against_oracle(R, B, E, shape):
     for x, d in zip(W, dev):
         got = d.view(torch.int16).cpu().numpy().view(np.uint16)
         np.testing.assert_array_equal(got, oracle.prefetch(slots, E, x))
+
+
+def gpu_reduce(slots, E, Gs):
+    dev = [torch.from_numpy(np.ascontiguousarray(g)).to(DEV) for g in Gs]
+    R, B = slots.shape
+    ep.ep_reduce_slot_grads(to_dev(slots), R, E, B, *dev)
+    torch.cuda.synchronize()
+    return [d.cpu().numpy() for d in dev]
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_reduce_slot_grads_against_oracle(seed):
+    rng = np.random.default_rng(seed)
+    R, B, E = 6, 3, 10
+    shape = (E + R * B, 7, 12)
+    Gs = [rng.standard_normal(shape).astype(np.float32) for _ in range(3)]
+    slots = rng.integers(-1, E, size=(R, B)).astype(np.int32)
+    slots[0, 0] = slots[1, 0] = slots[2, 2] = 4      # one expert, three slots
+    got = gpu_reduce(slots, E, Gs)
+    for g, G in zip(got, Gs):
+        np.testing.assert_array_equal(g, oracle.reduce_slot_grads(slots, E, G))
+
+
+def test_reduce_slot_grads_balanced_plan():
+    w = workloads.WORKLOADS["balanced"]
+    topk, _ = workloads.routing(w)
+    lay = gpu_layout(topk, w.R, w.S, w.E, 1)
+    g = compare(lay["counts"], w.R, w.S, w.K, w.B)
+    slots = g["slot_expert"]
+    assert (slots >= 0).sum() >= 1
+    rng = np.random.default_rng(5)
+    shape = (w.E + w.R * w.B, w.H, 16)               # narrow I for the test
+    Gs = [rng.standard_normal(shape).astype(np.float32) for _ in range(3)]
+    got = gpu_reduce(slots, w.E, Gs)
+    for gg, G in zip(got, Gs):
+        np.testing.assert_array_equal(gg, oracle.reduce_slot_grads(slots, w.E,
+                                                                   G))
+
+
+def test_reduce_slot_grads_rejects_large_tables():
+    t = torch.zeros(8, dtype=torch.float32, device=DEV)
+    s = torch.zeros(2048, dtype=torch.int32, device=DEV)
+    with pytest.raises(ep.EPError) as e:
+        ep.ep_reduce_slot_grads(s, 1024, 8, 2, t.view(1, 8).expand(2056, 8)
+                                .contiguous(), t.view(1, 8).expand(2056, 8)
+                                .contiguous(), t.view(1, 8).expand(2056, 8)
+                                .contiguous())
+    assert e.value.code == ep.EP_ERR_INVALID_ARG
