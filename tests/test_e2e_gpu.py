@@ -24,7 +24,8 @@ def test_round_trip(name):
     buf = EPBuffer(wl.S, wl.H, wl.K, wl.E, wl.R, token_padding=wl.pad,
                    fp8=wl.fp8)
     wd = to_dev(w)
-    recv, scales, recv_w, offsets = buf.dispatch(hid, wd, to_dev(topk))
+    recv, recv_w, offsets, handle = buf.dispatch(hid, wd, to_dev(topk))
+    scales = handle.recv_scales
     o = oracle.layout(topk, wl.E, wl.pad, buf.cap)
     np.testing.assert_array_equal(buf.pos.cpu().numpy(), o["pos"])
     np.testing.assert_array_equal(offsets.cpu().numpy(), o["offsets"])
@@ -35,7 +36,8 @@ def test_round_trip(name):
              scales[:used].repeat_interleave(128, dim=1)).to(torch.bfloat16)
     else:
         y = recv[:used]
-    out = buf.combine(y.contiguous(), wd)
+    out, gathered = buf.combine(handle, y.contiguous())
+    np.testing.assert_array_equal(gathered.cpu().numpy(), w)
     buf.check()
     x = hid.float()
     if wl.fp8:
