@@ -115,3 +115,15 @@ def test_large_batches_tma_path(N, K, H, rows):
     w = rng.standard_normal((N, K)).astype(np.float32)
     got = check(y, pos, w)
     assert np.all(got[7] == 0)
+
+
+def test_widest_row_and_k32():
+    rng = np.random.default_rng(11)
+    y = u16(workloads.bf16_normal((300, 32768), 12))
+    pos = rng.integers(0, 300, size=(40, 2)).astype(np.int32)
+    w = rng.random((40, 2)).astype(np.float32)
+    check(y, pos, w)
+    y = u16(workloads.bf16_normal((600, 1024), 13))
+    pos = rng.integers(0, 600, size=(2600, 32)).astype(np.int32)
+    w = rng.random((2600, 32)).astype(np.float32) / 32
+    check(y, pos, w)

@@ -142,3 +142,38 @@ def test_full_size_sampled(name):
         assert len(pad_rows) > 0
         sel = rows_to_host(d["recv"], pad_rows[:2000])
         assert np.all(sel == 0)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_k32(fp8):
+    topk, w, h = make(321, 2, 200, 32, 64, 256, distinct=True)
+    check_full(topk, w, h, 2, 200, 64, 256, 1, fp8=fp8)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_widest_row(fp8):
+    # H = 32768, the largest the ABI accepts: two input stages of 64 KB
+    topk, w, h = make(322, 1, 48, 3, 4, 32768)
+    check_full(topk, w, h, 1, 48, 4, 32768, 1, fp8=fp8)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_capacity_smaller_than_layout_is_reported(fp8):
+    # dispatch told about fewer rows than the layout used: rows past cap
+    # are skipped (never written) and EP_DEV_CAPACITY is raised
+    topk, w, h = make(323, 2, 100, 4, 8, 256)
+    g = gpu_layout(topk, 2, 100, 8, 1)
+    half = g["dev"]["cap"] // 2
+    g["dev"]["cap"] = half
+    d = gpu_dispatch(to_bf16_dev(h), w, g, 8, fp8)
+    assert d["status"] & 2                     # EP_DEV_CAPACITY
+    assert d["recv"].shape[0] == half
+    o = oracle.layout(topk, 8, 1)
+    keep = o["pos"] < half
+    rows = o["pos"][keep]
+    toks = np.nonzero(keep)[0]
+    if fp8:
+        q, s = oracle.quantize_rows(h)
+        np.testing.assert_array_equal(d["recv"].cpu().numpy()[rows], q[toks])
+    else:
+        np.testing.assert_array_equal(u16(d["recv"])[rows], h[toks])
