@@ -217,6 +217,19 @@ def traffic_from_profiles(kernel: str, workload: str, src_file: str):
 # the GPU path
 # --------------------------------------------------------------------------
 
+def layout_dispatch_kernels(wl, sms=148):
+    """Kernels one ep_layout_dispatch call launches, by the library's size
+    rule: one for N*K <= 32768 with at most 1024 entries per CTA; else the
+    cooperative layout kernel (tiles of 4096 entries all resident) or the
+    histogram + scan pair, then the dispatch kernel."""
+    entries = wl.N * wl.K
+    chunk = -(-wl.N // sms)
+    if entries <= 32768 and chunk * wl.K <= 1024:
+        return 1
+    tiles = -(-entries // 4096)
+    return (1 if tiles <= sms else 2) + 1
+
+
 class Path:
     """All device buffers of one replica, allocated once."""
 
@@ -265,7 +278,8 @@ class Path:
             rows = E + R * B
             self.W = [workloads.weight_buffer(rows, wl.H, wl.I, wl.seed + j,
                                               device=dev) for j in range(3)]
-        self.launches_per_step = 4 + (2 if wl.B > 0 else 0)
+        self.launches_per_step = (layout_dispatch_kernels(wl) + 1 +
+                                  (2 if wl.B > 0 else 0))
         self.backward = False
 
     def enable_backward(self, seed_offset=0):
@@ -327,6 +341,18 @@ class Path:
                                  p["slot"], self.status)
         self.ep.ep_prefetch_weights(p["slot"], wl.R, wl.E, wl.B, *self.W)
 
+    def layout_dispatch(self, io=None):
+        """The user's dispatch call: layout and copy (one launch for a small
+        batch, ep_layout + ep_dispatch otherwise)."""
+        wl = self.wl
+        io = io or self.io()
+        self.ep.ep_layout_dispatch(io["topk"], io["hidden"], io["w"], wl.R,
+                                   wl.S, wl.K, wl.E, wl.H, wl.pad, wl.fp8,
+                                   self.counts, self.offsets, self.pos,
+                                   self.row_src, self.recv, self.scales,
+                                   self.recv_w, workspace=self.ws,
+                                   status=self.status, cap=self.cap)
+
     def dispatch(self, io=None):
         wl = self.wl
         io = io or self.io()
@@ -342,10 +368,9 @@ class Path:
                            io["out"], status=self.status, cap=self.cap)
 
     def step(self, io=None):
-        self.layout(io)
+        self.layout_dispatch(io)
         if self.wl.B > 0:
             self.plan_prefetch()
-        self.dispatch(io)
         self.combine(io)
         if self.backward:
             self.combine_backward(io)
@@ -435,8 +460,8 @@ def run_gpu(args, wl):
         torch.cuda.synchronize()
     barrier()
     del graph
-    parts = {"layout": path.layout, "dispatch": path.dispatch,
-             "combine": path.combine}
+    parts = {"layout_dispatch": path.layout_dispatch, "layout": path.layout,
+             "dispatch": path.dispatch, "combine": path.combine}
     if wl.B > 0:
         parts["plan_prefetch"] = path.plan_prefetch
     if args.backward:
@@ -468,11 +493,19 @@ def run_gpu(args, wl):
         value = total_value_gbs(b_step, K, ws, ms_max)
         comb_gbs = b_com / (avg["combine"] * 1e-6) / 1e9
         dis_gbs = b_dis / (avg["dispatch"] * 1e-6) / 1e9
-        dom = "combine" if avg["combine"] >= avg["dispatch"] else "dispatch"
-        dom_bytes = b_com if dom == "combine" else b_dis
-        dom_gbs = comb_gbs if dom == "combine" else dis_gbs
-        kern = {"combine": ("k_combine", "combine.cu"),
-                "dispatch": ("k_dispatch", "dispatch.cu")}[dom]
+        ld_gbs = (b_lay + b_dis) / (avg["layout_dispatch"] * 1e-6) / 1e9
+        one_launch = layout_dispatch_kernels(wl) == 1
+        # the dominant kernel: combine, or the dispatch side's longest kernel
+        # (the single layout+dispatch kernel of a small batch)
+        if one_launch:
+            cand = ("layout_dispatch", "k_layout_small", "layout_small.cu",
+                    b_lay + b_dis, ld_gbs)
+        else:
+            cand = ("dispatch", "k_dispatch", "dispatch.cu", b_dis, dis_gbs)
+        if avg["combine"] >= avg[cand[0]]:
+            cand = ("combine", "k_combine", "combine.cu", b_com, comb_gbs)
+        dom, kname, ksrc, dom_bytes, dom_gbs = cand
+        kern = (kname, ksrc)
         src = os.path.join(ROOT, "combine_ep_layout_09_b200", "csrc", kern[1])
         traffic = traffic_from_profiles(kern[0], wl.name, src)
         clocks = clk.summary()
@@ -491,23 +524,30 @@ def run_gpu(args, wl):
             "data": "synthetic",
             "config": {
                 "workload": wl.describe,
-                "step": ("ep_layout + " + ("ep_plan_balanced + "
-                         "ep_prefetch_weights + " if wl.B else "") +
-                         "ep_dispatch + ep_combine" +
+                "step": ("ep_layout_dispatch (" +
+                         ("one launch" if one_launch else
+                          "ep_layout + ep_dispatch") + ") + " +
+                         ("ep_plan_balanced + ep_prefetch_weights + "
+                          if wl.B else "") + "ep_combine" +
                          (" + ep_combine_backward + ep_dispatch_backward"
                           if args.backward else "") +
                          (" + ep_reduce_slot_grads"
                           if args.backward and wl.B else "")),
                 "bytes_per_step": b_step,
                 "used_rows": used,
-                "l2": "no flush: every step moves >4 GB, inputs larger "
-                      "than the 126 MB L2",
+                "l2": (f"no flush: every step moves {b_step / 1e6:.0f} MB,"
+                       " more than the 126 MB L2" if b_step > 126e6 else
+                       "L2-resident: the step moves less than the 126 MB "
+                       "L2"),
                 "parallelism": f"{ws} independent replica(s), one per GPU",
                 "timing": "K steps captured in one CUDA graph, replayed "
                           "once, CUDA events around the replay; per-kernel "
                           "times from a graph of K launches of that kernel",
             },
             "breakdown": {
+                "layout_dispatch_us": round(med["layout_dispatch"], 2),
+                "layout_dispatch_GBps": round(ld_gbs, 1),
+                "layout_dispatch_one_launch": one_launch,
                 "layout_us": round(med["layout"], 2),
                 "dispatch_us": round(med["dispatch"], 2),
                 "combine_us": round(med["combine"], 2),
@@ -535,9 +575,11 @@ def run_gpu(args, wl):
                 "layout_bytes": b_lay, "prefetch_bytes": b_pre,
                 "frac_of_8TBps": {
                     "dispatch": round(dis_gbs / NOMINAL_HBM_GBS, 4),
+                    "layout_dispatch": round(ld_gbs / NOMINAL_HBM_GBS, 4),
                     "combine": round(comb_gbs / NOMINAL_HBM_GBS, 4)},
                 "frac_of_measured": {
                     "dispatch": round(dis_gbs / peak, 4),
+                    "layout_dispatch": round(ld_gbs / peak, 4),
                     "combine": round(comb_gbs / peak, 4)},
             },
             "roofline": {
@@ -556,8 +598,9 @@ def run_gpu(args, wl):
             "e2e": e2e,
             "gpu_launches": path.launches_per_step * K,
             "gpu_launches_note": "kernels of libeplayout.so in the timed "
-                                 "region; ep_layout adds one cudaMemsetAsync "
-                                 "per step",
+                                 "region" + ("" if one_launch else
+                                             "; ep_layout adds one "
+                                             "cudaMemsetAsync per step"),
         }
     if ws > 1:
         import torch.distributed as dist

@@ -81,6 +81,10 @@ def _declare(L):
     L.ep_dispatch.restype = i32
     L.ep_dispatch.argtypes = [P, P, P, P, P, i64, i32, i32, i32, i64, i32, P,
                               P, P, i32, P, P]
+    L.ep_layout_dispatch.restype = i32
+    L.ep_layout_dispatch.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32,
+                                     i32, P, P, P, P, i64, P, P, P, P, sz,
+                                     i32, P, P]
     L.ep_combine.restype = i32
     L.ep_combine.argtypes = [P, P, P, i64, i32, i32, i64, P, i32, P, P]
     L.ep_dispatch_backward.restype = i32
@@ -175,7 +179,7 @@ def ep_layout_workspace_bytes(num_tokens: int, K: int, E: int) -> int:
 def ep_layout(topk_experts, R, S, K, E, token_padding, tokens_per_expert,
               expert_offsets, pos, row_src, workspace, status=None,
               cap=None, stream=None):
-    """Histogram, padded expert offsets and stable positions (3 launches)."""
+    """Histogram, padded expert offsets and stable positions."""
     N = R * S
     cap = row_src.numel() if cap is None else int(cap)
     rc = lib().ep_layout(
@@ -214,6 +218,36 @@ def ep_dispatch(hidden, route_weights, pos, row_src, expert_offsets,
         _ptr(status, "status", _I32, 1, optional=True),
         _stream(stream))
     _check(rc, "ep_dispatch")
+
+
+def ep_layout_dispatch(topk_experts, hidden, route_weights, R, S, K, E, H,
+                       token_padding, fp8, tokens_per_expert, expert_offsets,
+                       pos, row_src, recv, recv_scales=None,
+                       recv_weights=None, workspace=None, num_sms=0,
+                       status=None, cap=None, stream=None):
+    """ep_layout then ep_dispatch; one launch for a small batch."""
+    N = R * S
+    cap = row_src.numel() if cap is None else int(cap)
+    rc = lib().ep_layout_dispatch(
+        _ptr(topk_experts, "topk_experts", _I32, N * K),
+        _ptr(hidden, "hidden", _BF16, N * H),
+        _ptr(route_weights, "route_weights", _F32, N * K),
+        R, S, K, E, H, token_padding, 1 if fp8 else 0,
+        _ptr(tokens_per_expert, "tokens_per_expert", _I32, E),
+        _ptr(expert_offsets, "expert_offsets", _I32, E + 1),
+        _ptr(pos, "pos", _I32, N * K),
+        _ptr(row_src, "row_src", _I32, cap),
+        cap,
+        _ptr(recv, "recv", _FP8 if fp8 else _BF16, cap * H),
+        _ptr(recv_scales, "recv_scales", _F32, cap * (H // 128),
+             optional=not fp8),
+        _ptr(recv_weights, "recv_weights", _F32, cap, optional=True),
+        _ptr(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(),
+        int(num_sms),
+        _ptr(status, "status", _I32, 1, optional=True),
+        _stream(stream))
+    _check(rc, "ep_layout_dispatch")
 
 
 def ep_combine(expert_out, pos, route_weights, num_tokens, K, H, out,

@@ -107,14 +107,13 @@ class EPBuffer:
         FP8 scales are handle.recv_scales."""
         self.index = (self.index + 1) % len(self.sets)   # idx ^= 1
         st = self.sets[self.index]
-        B.ep_layout(topk_experts_sk, self.R, self.S, self.K, self.E, self.pad,
-                    st.tokens_per_expert, st.expert_offsets, st.pos,
-                    st.row_src, self.workspace, self.status, cap=self.cap,
-                    stream=stream)
-        B.ep_dispatch(hidden_sh, route_weights_sk, st.pos, st.row_src,
-                      st.expert_offsets, self.N, self.K, self.E, self.H,
-                      self.fp8, st.recv, st.recv_scales, st.recv_weights,
-                      self.num_sms, self.status, cap=self.cap, stream=stream)
+        B.ep_layout_dispatch(topk_experts_sk, hidden_sh, route_weights_sk,
+                             self.R, self.S, self.K, self.E, self.H, self.pad,
+                             self.fp8, st.tokens_per_expert,
+                             st.expert_offsets, st.pos, st.row_src, st.recv,
+                             st.recv_scales, st.recv_weights, self.workspace,
+                             self.num_sms, self.status, cap=self.cap,
+                             stream=stream)
         h = DispatchHandle(self.index, st.tokens_per_expert,
                            st.expert_offsets, st.pos, st.row_src, st.recv,
                            st.recv_scales, st.recv_weights)

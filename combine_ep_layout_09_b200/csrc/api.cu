@@ -8,7 +8,7 @@
 
 namespace {
 
-constexpr int kAbiVersion = 2;
+constexpr int kAbiVersion = 3;
 constexpr int kMaxK = 32;
 constexpr int kMaxH = 32768;
 constexpr int64_t kMaxEntries = (int64_t(1) << 30) - 1;
@@ -100,10 +100,62 @@ int ep_layout(const int32_t* topk_experts, int R, int S, int K, int E,
     return EP_ERR_ALIGNMENT;
   if (cap > 0 && !aligned16(row_src)) return EP_ERR_ALIGNMENT;
   if (workspace_bytes < ep::layout_workspace_bytes(M, E)) return EP_ERR_WORKSPACE;
+  const int sms = sms_or_all(0);
+  if (ep::small_layout_fits(N, K, E, 8, 0, sms))
+    return cuda_rc(ep::launch_layout_small(topk_experts, N, K, E, token_padding,
+                                           tokens_per_expert, expert_offsets,
+                                           pos, row_src, cap, sms, status,
+                                           as_stream(stream)));
   return cuda_rc(ep::launch_layout(topk_experts, M, E, token_padding,
                                    tokens_per_expert, expert_offsets, pos,
-                                   row_src, cap, workspace, status,
-                                   sms_or_all(0), as_stream(stream)));
+                                   row_src, cap, workspace, status, sms,
+                                   as_stream(stream)));
+}
+
+int ep_layout_dispatch(const int32_t* topk_experts, const void* hidden,
+                       const float* route_weights, int R, int S, int K, int E,
+                       int H, int token_padding, int fp8,
+                       int32_t* tokens_per_expert, int32_t* expert_offsets,
+                       int32_t* pos, int32_t* row_src, int64_t cap, void* recv,
+                       float* recv_scales, float* recv_weights,
+                       void* workspace, size_t workspace_bytes, int num_sms,
+                       int32_t* status, void* stream) {
+  if (R < 1 || S < 0 || K < 1 || K > kMaxK || E < 1 || E > ep::kMaxExperts ||
+      E % R != 0 || token_padding < 1 || H < 8 || H > kMaxH || H % 8 != 0 ||
+      (fp8 != 0 && fp8 != 1) || (fp8 && H % 128 != 0) || num_sms < 0)
+    return EP_ERR_INVALID_ARG;
+  const int64_t N = int64_t(R) * S;
+  const int64_t M = N * K;
+  if (M > kMaxEntries) return EP_ERR_INVALID_ARG;
+  const int64_t bound = ep_capacity_bound(N, K, E, token_padding);
+  if (cap < bound || cap > INT32_MAX) return EP_ERR_CAPACITY;
+  if (!aligned16(tokens_per_expert) || !aligned16(expert_offsets) ||
+      !aligned16(workspace) || !status_ok(status))
+    return EP_ERR_ALIGNMENT;
+  if (M > 0 && (!aligned16(topk_experts) || !aligned16(pos) ||
+                !aligned16(hidden) || !aligned16(route_weights)))
+    return EP_ERR_ALIGNMENT;
+  if (cap > 0 && (!aligned16(row_src) || !aligned16(recv))) return EP_ERR_ALIGNMENT;
+  if (cap > 0 && fp8 && !aligned16(recv_scales)) return EP_ERR_ALIGNMENT;
+  if (recv_weights && !aligned16(recv_weights)) return EP_ERR_ALIGNMENT;
+  if (workspace_bytes < ep::layout_workspace_bytes(M, E)) return EP_ERR_WORKSPACE;
+  const int sms = sms_or_all(num_sms);
+  cudaStream_t st = as_stream(stream);
+  if (ep::small_layout_fits(N, K, E, H, fp8 ? 2 : 1, sms))
+    return cuda_rc(ep::launch_layout_dispatch_small(
+        topk_experts, N, K, E, token_padding, H, fp8 != 0, tokens_per_expert,
+        expert_offsets, pos, row_src, cap, hidden, route_weights, recv,
+        fp8 ? recv_scales : nullptr, recv_weights, sms, status, st));
+  cudaError_t err = ep::launch_layout(topk_experts, M, E, token_padding,
+                                      tokens_per_expert, expert_offsets, pos,
+                                      row_src, cap, workspace, status,
+                                      sms_or_all(0), st);
+  if (err != cudaSuccess) return EP_ERR_CUDA;
+  if (N == 0 && cap == 0) return EP_OK;
+  return cuda_rc(ep::launch_dispatch(hidden, route_weights, pos, row_src,
+                                     expert_offsets, N, K, E, H, cap, fp8 != 0,
+                                     recv, fp8 ? recv_scales : nullptr,
+                                     recv_weights, sms, status, st));
 }
 
 int ep_dispatch(const void* hidden, const float* route_weights,

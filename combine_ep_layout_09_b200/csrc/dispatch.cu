@@ -22,22 +22,12 @@
 //                    in shared memory (codes, then the row's scales); one
 //                    thread bulk-stores that stage K times.
 //
-// Quantisation ("bracketed reciprocal"): the code must be e4m3(RN(x/s)) with
-// the fp32 quotient correctly rounded. With inv = RN(1/s), the products
-// lo = RN(x * RN(inv*(1-2^-20))) and hi = RN(x * RN(inv*(1+2^-20))) enclose
-// RN(x/s) (each rounding moves a value by at most 2^-24 relative, far
-// inside the 2^-20 margin). Rounding to E4M3 is monotone, so when lo and hi
-// encode to the same code that code is e4m3(RN(x/s)). Otherwise the pair is
-// recomputed with the correctly rounded division __fdiv_rn. That happens
-// for about 3e-5 of the values, the ones within 2^-20 of a rounding
-// boundary. Values in the fp32 subnormal range all encode to +-0 on the
-// correct side, so the bracket needs no normal-range assumption there. A
-// scale below 2^-125, whose reciprocal could overflow, takes the division
-// path for the whole group.
+// The E4M3 quantiser and its exactness argument are in ep_quant.cuh.
 #include <algorithm>
 
 #include "ep_device.cuh"
 #include "ep_launch.h"
+#include "ep_quant.cuh"
 
 namespace ep {
 namespace {
@@ -52,72 +42,6 @@ __host__ __device__ constexpr uint32_t align128(uint32_t x) {
 
 __device__ __forceinline__ void named_barrier(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-// ---------------------------------------------------------------------------
-// E4M3 quantisation of 16 values by one group scale (shared with the
-// diagnostic entry point so that the tests exercise this exact code)
-// ---------------------------------------------------------------------------
-
-struct GroupScale {
-  float scale;   // the group's fp32 scale
-  float inv_lo;  // RN(RN(1/scale) * (1 - 2^-20))
-  float inv_hi;  // RN(RN(1/scale) * (1 + 2^-20))
-  bool bracket;  // reciprocal path valid (scale >= 2^-125)
-};
-
-__device__ __forceinline__ GroupScale make_group_scale(float scale) {
-  GroupScale g;
-  g.scale = scale;
-  g.bracket = scale >= 0x1p-125f;
-  const float inv = g.bracket ? __frcp_rn(scale) : 0.0f;
-  g.inv_lo = inv * (1.0f - 0x1p-20f);
-  g.inv_hi = inv * (1.0f + 0x1p-20f);
-  return g;
-}
-
-// Two codes (low byte = a) for e4m3(RN(a/scale)), e4m3(RN(b/scale)).
-__device__ __forceinline__ uint32_t codes2_exact(float a, float b,
-                                                 const GroupScale& g) {
-  return e4m3x2(__fdiv_rn(a, g.scale), __fdiv_rn(b, g.scale));
-}
-
-// 16 codes of x[0..15] (scale != 0); bytes in channel order.
-__device__ __forceinline__ uint4 quantize16(const float (&x)[16],
-                                            const GroupScale& g) {
-  uint32_t c[8];
-  bool agree = g.bracket;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t lo = e4m3x2(x[2 * i] * g.inv_lo, x[2 * i + 1] * g.inv_lo);
-    const uint32_t hi = e4m3x2(x[2 * i] * g.inv_hi, x[2 * i + 1] * g.inv_hi);
-    agree = agree && (lo == hi);
-    c[i] = lo;
-  }
-  if (!agree) {  // rare: some value sits on a rounding boundary
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t lo = e4m3x2(x[2 * i] * g.inv_lo, x[2 * i + 1] * g.inv_lo);
-      const uint32_t hi = e4m3x2(x[2 * i] * g.inv_hi, x[2 * i + 1] * g.inv_hi);
-      if (!g.bracket || lo != hi) c[i] = codes2_exact(x[2 * i], x[2 * i + 1], g);
-    }
-  }
-  return make_uint4(c[0] | (c[1] << 16), c[2] | (c[3] << 16),
-                    c[4] | (c[5] << 16), c[6] | (c[7] << 16));
-}
-
-// Unpack 16 bf16 (two 16-byte words) to fp32; returns max |x|.
-__device__ __forceinline__ float unpack16(const uint4& a, const uint4& b,
-                                          float (&x)[16]) {
-  const uint32_t wd[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    x[2 * i] = bf16_lo(wd[i]);
-    x[2 * i + 1] = bf16_hi(wd[i]);
-    amax = fmaxf(amax, fmaxf(fabsf(x[2 * i]), fabsf(x[2 * i + 1])));
-  }
-  return amax;
 }
 
 // ---------------------------------------------------------------------------
@@ -333,24 +257,9 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32)
       for (int u = warp; u * kUnitCh < H; u += cw) {
         const int c0 = u * kUnitCh + lane * 16;  // first channel of this lane
         const bool act = c0 < H;                 // H % 128 == 0: whole groups
-        uint4 a = make_uint4(0u, 0u, 0u, 0u), b = a;
-        if (act && ok) {
-          a = *reinterpret_cast<const uint4*>(row + size_t(c0) * 2);
-          b = *reinterpret_cast<const uint4*>(row + size_t(c0) * 2 + 16);
-        }
-        float x[16];
-        float amax = unpack16(a, b, x);
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-        const float scale = __fdiv_rn(amax, 448.0f);
-        uint4 q = make_uint4(0u, 0u, 0u, 0u);
-        if (scale != 0.0f) q = quantize16(x, make_group_scale(scale));
-        if (act) {
-          *reinterpret_cast<uint4*>(out + c0) = q;
-          if (bulk_scales && (lane & 7) == 0)
-            reinterpret_cast<float*>(out + H)[c0 >> 7] = scale;
-        }
+        const float scale = quantize_lane16(row, out, c0, act && ok);
+        if (act && bulk_scales && (lane & 7) == 0)
+          reinterpret_cast<float*>(out + H)[c0 >> 7] = scale;
         if (!bulk_scales) {
           // lanes store their group's scale to every destination row
           for (int k = 0; k < K; ++k) {

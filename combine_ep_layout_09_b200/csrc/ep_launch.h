@@ -24,6 +24,31 @@ cudaError_t launch_layout(const int32_t* topk, int64_t entries, int E, int pad,
                           void* workspace, int32_t* status, int num_sms,
                           cudaStream_t stream);
 
+// Small batches: one launch, every CTA counts all entries itself and places
+// its own chunk of tokens (layout_small.cu). Taken up to kSmallMaxEntries
+// entries N*K, with at most kSmallMaxChunkEntries entries ranked per CTA and
+// the CTA's shared-memory plan within kSmallMaxSmem bytes.
+constexpr int64_t kSmallMaxEntries = 32768;
+constexpr int64_t kSmallMaxChunkEntries = 1024;
+constexpr int kSmallMaxSmem = 227 * 1024;
+
+// copy: 0 layout only, 1 bf16 rows, 2 FP8 rows
+bool small_layout_fits(int64_t N, int K, int E, int H, int copy, int num_sms);
+
+cudaError_t launch_layout_small(const int32_t* topk, int64_t N, int K, int E,
+                                int pad, int32_t* tokens_per_expert,
+                                int32_t* expert_offsets, int32_t* pos,
+                                int32_t* row_src, int64_t cap, int num_sms,
+                                int32_t* status, cudaStream_t stream);
+
+// ep_layout followed by ep_dispatch, in one launch
+cudaError_t launch_layout_dispatch_small(
+    const int32_t* topk, int64_t N, int K, int E, int pad, int H, bool fp8,
+    int32_t* tokens_per_expert, int32_t* expert_offsets, int32_t* pos,
+    int32_t* row_src, int64_t cap, const void* hidden, const float* w,
+    void* recv, float* scales, float* recv_w, int num_sms, int32_t* status,
+    cudaStream_t stream);
+
 // ---- dispatch / combine ---------------------------------------------------
 
 cudaError_t launch_dispatch(const void* hidden, const float* w,

@@ -31,6 +31,7 @@
 //              in arrival order.
 #include <algorithm>
 
+#include "ep_block.cuh"
 #include "ep_device.cuh"
 #include "ep_launch.h"
 
@@ -64,125 +65,6 @@ static_assert(sizeof(WsHeader) == 256, "header size");
 
 constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// In-place exclusive scan of buf[0..n) (shared memory) by a CTA of THREADS
-// threads; each thread owns a contiguous run. Returns the total.
-template <int THREADS>
-__device__ int32_t block_exclusive_scan(int32_t* buf, int n, int32_t* warp_tmp) {
-  static_assert(THREADS / 32 <= 32, "one warp scans the warp sums");
-  const int per = (n + THREADS - 1) / THREADS;
-  const int lo = min(n, int(threadIdx.x) * per);
-  const int hi = min(lo + per, n);
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  int32_t local = 0;
-  for (int i = lo; i < hi; ++i) local += buf[i];
-  int32_t x = local;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) warp_tmp[wid] = x;
-  __syncthreads();
-  if (wid == 0) {
-    int32_t s = lane < THREADS / 32 ? warp_tmp[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int32_t y = __shfl_up_sync(0xffffffffu, s, o);
-      if (lane >= o) s += y;
-    }
-    if (lane < THREADS / 32) warp_tmp[lane] = s;
-  }
-  __syncthreads();
-  int32_t run = x - local + (wid > 0 ? warp_tmp[wid - 1] : 0);
-  const int32_t total = warp_tmp[THREADS / 32 - 1];
-  for (int i = lo; i < hi; ++i) {
-    const int32_t v = buf[i];
-    buf[i] = run;
-    run += v;
-  }
-  __syncthreads();
-  return total;
-}
-
-// Two in-place exclusive scans at once (a and b, n values each, shared
-// memory); totals returned through ta / tb.
-template <int THREADS>
-__device__ void block_exclusive_scan2(int32_t* a, int32_t* b, int n,
-                                      int32_t* warp_tmp /* [2*THREADS/32] */,
-                                      int32_t& ta, int32_t& tb) {
-  constexpr int W = THREADS / 32;
-  const int per = (n + THREADS - 1) / THREADS;
-  const int lo = min(n, int(threadIdx.x) * per);
-  const int hi = min(lo + per, n);
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  int32_t la = 0, lb = 0;
-  for (int i = lo; i < hi; ++i) {
-    la += a[i];
-    lb += b[i];
-  }
-  int32_t xa = la, xb = lb;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int32_t ya = __shfl_up_sync(0xffffffffu, xa, o);
-    const int32_t yb = __shfl_up_sync(0xffffffffu, xb, o);
-    if (lane >= o) {
-      xa += ya;
-      xb += yb;
-    }
-  }
-  if (lane == 31) {
-    warp_tmp[wid] = xa;
-    warp_tmp[W + wid] = xb;
-  }
-  __syncthreads();
-  if (wid == 0) {
-    int32_t sa = lane < W ? warp_tmp[lane] : 0;
-    int32_t sb = lane < W ? warp_tmp[W + lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int32_t ya = __shfl_up_sync(0xffffffffu, sa, o);
-      const int32_t yb = __shfl_up_sync(0xffffffffu, sb, o);
-      if (lane >= o) {
-        sa += ya;
-        sb += yb;
-      }
-    }
-    if (lane < W) {
-      warp_tmp[lane] = sa;
-      warp_tmp[W + lane] = sb;
-    }
-  }
-  __syncthreads();
-  int32_t ra = xa - la + (wid > 0 ? warp_tmp[wid - 1] : 0);
-  int32_t rb = xb - lb + (wid > 0 ? warp_tmp[W + wid - 1] : 0);
-  ta = warp_tmp[W - 1];
-  tb = warp_tmp[2 * W - 1];
-  for (int i = lo; i < hi; ++i) {
-    const int32_t va = a[i], vb = b[i];
-    a[i] = ra;
-    b[i] = rb;
-    ra += va;
-    rb += vb;
-  }
-  __syncthreads();
-}
-
-// Bits that tell the experts [0, E) apart.
-__device__ __forceinline__ int expert_bits(int E) {
-  return E <= 1 ? 0 : 32 - __clz(E - 1);
-}
-
-// Lanes of the warp whose key equals this lane's key (valid keys >= 0 only;
-// the result is meaningless for invalid lanes). One ballot per key bit.
-__device__ __forceinline__ unsigned same_key_lanes(int key, int nbits) {
-  unsigned peers = __ballot_sync(0xffffffffu, key >= 0);
-  for (int b = 0; b < nbits; ++b) {
-    const bool bit = (key >> b) & 1;
-    const unsigned bal = __ballot_sync(0xffffffffu, bit);
-    peers &= bit ? bal : ~bal;
-  }
-  return peers;
-}
 
 __global__ void __launch_bounds__(kHistThreads)
     k_histogram(const int32_t* __restrict__ topk, int64_t M, int E, int pad,

@@ -58,7 +58,7 @@ extern "C" {
 #define EP_DEV_SLOTS 8       /* the balanced plan needed more than B slots on a rank */
 #define EP_DEV_PLAN_TOTAL 16 /* sum(tokens_per_expert) != R*S*K; plan not written */
 
-/* Version of this ABI (bumped on any signature change). */
+/* Version of this ABI (bumped when an entry point is added or changed). */
 EP_API int ep_abi_version(void);
 
 /* Static text for a return code or a single status bit. */
@@ -102,7 +102,11 @@ EP_API size_t ep_layout_workspace_bytes(int64_t num_tokens, int K, int E);
  *                        shared by two calls in flight at the same time
  *      status            device int32, EP_DEV_BAD_EXPERT / EP_DEV_TIMEOUT /
  *                        EP_DEV_CAPACITY may be OR-ed in
- * Three launches (one memset, two kernels) on `stream`.
+ * Launches on `stream`: for N*K <= 32768 (and at most 1024 entries per
+ * SM) one kernel in which every CTA counts all entries and places its own
+ * tokens, workspace unused; above that a memset and one cooperative kernel
+ * (a decoupled look-back scan), or a memset and two kernels when the tiles
+ * cannot all be resident.
  */
 EP_API int ep_layout(const int32_t* topk_experts, int R, int S, int K, int E,
               int token_padding, int32_t* tokens_per_expert,
@@ -175,6 +179,39 @@ EP_API int ep_dispatch(const void* hidden, const float* route_weights,
                 int E, int H, int64_t cap, int fp8, void* recv,
                 float* recv_scales, float* recv_weights, int num_sms,
                 int32_t* status, void* stream);
+
+/*
+ * ep_layout_dispatch -- ep_layout then ep_dispatch, in ONE launch for small
+ * (decode-sized) batches ("DeepSeek开源周第二天：DeepEP深度分析", "DeepEP介绍":
+ * low-latency kernels for latency-sensitive decoding). Every CTA counts all
+ * N*K entries in shared memory, places its own contiguous chunk of tokens
+ * and copies their rows, with no workspace and no wait on another CTA.
+ * Taken when N*K <= 32768, at most 1024 entries fall to one CTA and the
+ * CTA's staged rows fit in shared memory; otherwise the call runs ep_layout
+ * and ep_dispatch as separate launches. Either way the results are those of
+ * the two calls, bit for bit.
+ *
+ * in   topk_experts, R, S, K, E, token_padding, cap, workspace,
+ *      workspace_bytes   as for ep_layout (the workspace is needed only when
+ *                        the batch is too large for the single launch)
+ *      hidden, route_weights, H, fp8, num_sms
+ *                        as for ep_dispatch
+ * out  tokens_per_expert, expert_offsets, pos, row_src
+ *                        as for ep_layout
+ *      recv, recv_scales, recv_weights
+ *                        as for ep_dispatch
+ *      status            any bit ep_layout or ep_dispatch may set
+ * Errors: those of ep_layout and ep_dispatch, checked before any launch.
+ */
+EP_API int ep_layout_dispatch(const int32_t* topk_experts, const void* hidden,
+                              const float* route_weights, int R, int S, int K,
+                              int E, int H, int token_padding, int fp8,
+                              int32_t* tokens_per_expert,
+                              int32_t* expert_offsets, int32_t* pos,
+                              int32_t* row_src, int64_t cap, void* recv,
+                              float* recv_scales, float* recv_weights,
+                              void* workspace, size_t workspace_bytes,
+                              int num_sms, int32_t* status, void* stream);
 
 /*
  * ep_combine -- gather each token's K expert outputs and reduce them with the

@@ -115,3 +115,45 @@ def rows_to_host(t: torch.Tensor, rows: np.ndarray) -> np.ndarray:
     if sel.dtype in (torch.uint8, torch.float8_e4m3fn):
         return sel.view(torch.uint8).cpu().numpy()
     return sel.cpu().numpy()
+
+
+def gpu_layout_dispatch(topk: np.ndarray, hidden_dev: torch.Tensor,
+                        w: np.ndarray, R: int, S: int, E: int, pad: int,
+                        fp8: bool, num_sms: int = 0, with_weights: bool = True,
+                        cap: int | None = None):
+    """ep_layout_dispatch with sentinel-filled outputs (garbage workspace)."""
+    N, K = topk.shape
+    H = hidden_dev.shape[1]
+    if cap is None:
+        cap = ep.ep_capacity_bound(N, K, E, pad)
+    rows = max(cap, 1)
+    i32 = dict(dtype=torch.int32, device=DEV)
+    counts = torch.full((E,), -9, **i32)
+    offsets = torch.full((E + 1,), -9, **i32)
+    pos = torch.full((max(N, 1), K), -9, **i32)
+    row_src = torch.full((rows,), ROW_SRC_FILL, **i32)
+    if fp8:
+        recv = torch.full((rows, H), RECV_FP8_FILL, dtype=torch.uint8,
+                          device=DEV)
+        scales = torch.full((rows, H // 128), SCALE_FILL,
+                            dtype=torch.float32, device=DEV)
+    else:
+        recv = torch.full((rows, H), RECV_BF16_FILL, dtype=torch.int16,
+                          device=DEV).view(torch.bfloat16)
+        scales = None
+    recv_w = torch.full((rows,), RECV_W_FILL, dtype=torch.float32,
+                        device=DEV) if with_weights else None
+    wsb = ep.ep_layout_workspace_bytes(N, K, E)
+    ws = torch.randint(0, 255, (max(wsb, 16),), dtype=torch.uint8,
+                       device=DEV)
+    st = status_tensor()
+    t = to_dev(topk.astype(np.int32) if N > 0 else np.zeros((1, K), np.int32))
+    wd = to_dev(w.astype(np.float32) if N > 0 else np.zeros((1, K), np.float32))
+    ep.ep_layout_dispatch(t, hidden_dev, wd, R, S, K, E, H, pad, fp8, counts,
+                          offsets, pos, row_src, recv, scales, recv_w,
+                          workspace=ws, num_sms=num_sms, status=st, cap=cap)
+    torch.cuda.synchronize()
+    return dict(counts=counts.cpu().numpy(), offsets=offsets.cpu().numpy(),
+                pos=pos[:N].cpu().numpy(), row_src=row_src[:cap].cpu().numpy(),
+                recv=recv, scales=scales, recv_w=recv_w,
+                status=int(st[0].item()), cap=cap)

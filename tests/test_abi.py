@@ -41,7 +41,7 @@ def test_library_is_the_in_tree_build():
 
 
 def test_pure_host_entry_points():
-    assert ep.ep_abi_version() == 2
+    assert ep.ep_abi_version() == 3
     assert ep.ep_capacity_bound(32768, 8, 256, 128) == 32768 * 8 + 256 * 127
     assert ep.ep_capacity_bound(10, 2, 4, 1) == 20
     assert ep.ep_capacity_bound(-1, 2, 4, 1) < 0
@@ -106,6 +106,34 @@ def test_dispatch_combine_reject_on_host():
                           None) == ep.EP_ERR_ALIGNMENT
     assert lib.ep_combine(ok, ok, ok, 0, 2, 16, 16, ok, 0, None,
                           None) == ep.EP_OK                # nothing to do
+
+
+def test_layout_dispatch_rejects_on_host():
+    lib = _raw()
+    P, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    lib.ep_layout_dispatch.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32,
+                                       i32, P, P, P, P, i64, P, P, P, P, sz,
+                                       i32, P, P]
+    ok = ctypes.c_void_p(1 << 20)
+    bad = ctypes.c_void_p((1 << 20) + 8)
+    args = dict(R=4, S=8, K=2, E=8, H=256, pad=1, fp8=0, cap=64, recv=ok,
+                scales=ok, ws=1 << 20, sms=0)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.ep_layout_dispatch(ok, ok, ok, a["R"], a["S"], a["K"],
+                                      a["E"], a["H"], a["pad"], a["fp8"], ok,
+                                      ok, ok, ok, a["cap"], a["recv"],
+                                      a["scales"], None, ok, a["ws"],
+                                      a["sms"], None, None)
+    assert call(E=10) == ep.EP_ERR_INVALID_ARG        # E % R != 0
+    assert call(fp8=1, H=200) == ep.EP_ERR_INVALID_ARG
+    assert call(H=12) == ep.EP_ERR_INVALID_ARG
+    assert call(sms=-1) == ep.EP_ERR_INVALID_ARG
+    assert call(cap=63) == ep.EP_ERR_CAPACITY
+    assert call(recv=bad) == ep.EP_ERR_ALIGNMENT
+    assert call(fp8=1, scales=None) == ep.EP_ERR_ALIGNMENT
+    assert call(ws=0) == ep.EP_ERR_WORKSPACE
 
 
 def test_plan_prefetch_reject_on_host():
