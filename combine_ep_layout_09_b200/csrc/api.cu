@@ -155,7 +155,7 @@ int ep_layout_dispatch(const int32_t* topk_experts, const void* hidden,
   return cuda_rc(ep::launch_dispatch(hidden, route_weights, pos, row_src,
                                      expert_offsets, N, K, E, H, cap, fp8 != 0,
                                      recv, fp8 ? recv_scales : nullptr,
-                                     recv_weights, sms, status, st));
+                                     recv_weights, sms, status, st, true));
 }
 
 int ep_dispatch(const void* hidden, const float* route_weights,

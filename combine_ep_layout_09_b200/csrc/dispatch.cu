@@ -111,6 +111,7 @@ __global__ void __launch_bounds__(32)
     }
   }
   __syncwarp();
+  grid_dependency_wait();  // pos / row_src / offsets may come from the layout
 
   bool ok = true;
   for (int64_t i = 0; i < n_mine && ok; ++i) {
@@ -231,6 +232,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32)
   } else {
     // ---- consumers --------------------------------------------------------
     const bool issuer = (warp == 0 && lane == 0);
+    grid_dependency_wait();  // pos may come from the layout kernel ahead
     int it = 0;
     for (int64_t t = blockIdx.x; t < N; t += gridDim.x, ++it) {
       const int s = it % s_in;
@@ -300,6 +302,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32)
     }
     if (issuer) bulk_wait_all<0>();
   }
+  grid_dependency_wait();  // row_src / offsets may come from the layout
   __syncthreads();
   zero_padding_rows<true>(row_src, offsets, E, H, cap, recv, scales, recv_w);
 }
@@ -359,7 +362,7 @@ cudaError_t launch_dispatch(const void* hidden, const float* w,
                             const int32_t* expert_offsets, int64_t N, int K,
                             int E, int H, int64_t cap, bool fp8, void* recv,
                             float* recv_scales, float* recv_w, int num_sms,
-                            int32_t* status, cudaStream_t stream) {
+                            int32_t* status, cudaStream_t stream, bool pdl) {
   const Cfg c = fp8 ? fp8_cfg(H) : bf16_cfg(H);
   const void* kern = fp8 ? reinterpret_cast<const void*>(k_dispatch_fp8)
                          : reinterpret_cast<const void*>(k_dispatch_bf16);
@@ -377,15 +380,26 @@ cudaError_t launch_dispatch(const void* hidden, const float* w,
                            std::max<int64_t>(N, (cap + 31) / 32)));
   const uint16_t* h = static_cast<const uint16_t*>(hidden);
   uint8_t* r = static_cast<uint8_t*>(recv);
+  // With pdl the launch may begin while the kernel ahead of it (the layout
+  // that wrote pos / row_src / offsets) is still running; the kernels wait
+  // for it before reading those.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(grid));
+  cfg.blockDim = dim3(unsigned(c.threads));
+  cfg.dynamicSmemBytes = c.smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
   if (fp8)
-    k_dispatch_fp8<<<int(grid), c.threads, c.smem, stream>>>(
-        h, w, pos, row_src, expert_offsets, N, K, E, H, cap, r, recv_scales,
-        recv_w, c.s_in, c.s_out, status);
-  else
-    k_dispatch_bf16<<<int(grid), c.threads, c.smem, stream>>>(
-        h, w, pos, row_src, expert_offsets, N, K, E, H, cap, r, recv_w,
-        c.s_in, status);
-  return cudaGetLastError();
+    return cudaLaunchKernelEx(&cfg, k_dispatch_fp8, h, w, pos, row_src,
+                              expert_offsets, N, K, E, H, cap, r, recv_scales,
+                              recv_w, c.s_in, c.s_out, status);
+  return cudaLaunchKernelEx(&cfg, k_dispatch_bf16, h, w, pos, row_src,
+                            expert_offsets, N, K, E, H, cap, r, recv_w, c.s_in,
+                            status);
 }
 
 cudaError_t launch_debug_quantize(const float* x, const float* scale,

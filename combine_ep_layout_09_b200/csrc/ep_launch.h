@@ -56,7 +56,8 @@ cudaError_t launch_dispatch(const void* hidden, const float* w,
                             const int32_t* expert_offsets, int64_t N, int K,
                             int E, int H, int64_t cap, bool fp8, void* recv,
                             float* recv_scales, float* recv_w, int num_sms,
-                            int32_t* status, cudaStream_t stream);
+                            int32_t* status, cudaStream_t stream,
+                            bool pdl = false);
 
 // w == NULL: unit weights (dispatch backward)
 cudaError_t launch_combine(const void* y, const int32_t* pos, const float* w,

@@ -434,6 +434,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                      int num_tiles, int32_t* __restrict__ pos,
                      int32_t* __restrict__ row_src, int64_t cap,
                      int32_t* __restrict__ status) {
+  grid_launch_dependents();
   extern __shared__ int32_t smem[];
   ScanSmem sm(smem, E);
   __shared__ int s_tile;
@@ -470,6 +471,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                    int32_t* __restrict__ expert_offsets,
                    int32_t* __restrict__ pos, int32_t* __restrict__ row_src,
                    int64_t cap, int32_t* __restrict__ status) {
+  grid_launch_dependents();
   extern __shared__ int32_t smem[];
   ScanSmem sm(smem, E);
   __shared__ int32_t s_warp2[2 * kScanThreads / 32];

@@ -188,8 +188,10 @@ EP_API int ep_dispatch(const void* hidden, const float* route_weights,
  * and copies their rows, with no workspace and no wait on another CTA.
  * Taken when N*K <= 32768, at most 1024 entries fall to one CTA and the
  * CTA's staged rows fit in shared memory; otherwise the call runs ep_layout
- * and ep_dispatch as separate launches. Either way the results are those of
- * the two calls, bit for bit.
+ * and ep_dispatch as separate launches, the dispatch kernel launched as a
+ * programmatic dependent of the layout kernel (its CTAs start loading token
+ * rows while the layout finishes). Either way the results are those of the
+ * two calls, bit for bit.
  *
  * in   topk_experts, R, S, K, E, token_padding, cap, workspace,
  *      workspace_bytes   as for ep_layout (the workspace is needed only when
