@@ -20,7 +20,7 @@
 // agree with it on every bit. The cost is the same whatever the keys, unlike
 // a hardware match whose cost grows with the number of distinct keys.
 //
-// Two paths:
+// Two paths here (small batches, N*K <= 32768, take layout_small.cu instead):
 //   fused      (tiles fit co-resident) one cooperative launch: the last tile's
 //              inclusive prefix holds every expert's total; every tile reads
 //              it, scans the padded totals into the expert offsets itself,

@@ -162,3 +162,17 @@ def test_widest_rows_single_stage_ring(fp8):
     R, S, K, E, H = 1, 8, 4, 8, 32768
     topk, w, h = make(13, R * S, K, E, H, distinct=True)
     check(topk, w, h, R, S, E, 2, fp8, num_sms=2)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_duplicate_ids_single_expert_and_wide_padding(fp8):
+    # ids repeat inside a token (K > E), one expert takes every entry, and
+    # a padding of 1000 rows per expert dwarfs the batch
+    R, S, K, E, H = 2, 60, 4, 2, 256
+    rng = np.random.default_rng(17)
+    topk = rng.integers(0, E, size=(R * S, K)).astype(np.int32)
+    w = rng.random((R * S, K)).astype(np.float32)
+    h = u16(workloads.bf16_normal((R * S, H), 17).to(torch.bfloat16))
+    check(topk, w, h, R, S, E, 1, fp8)
+    check(np.full((R * S, K), 1, np.int32), w, h, R, S, E, 7, fp8)
+    check(topk, w, h, R, S, E, 1000, fp8)
