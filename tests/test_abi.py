@@ -159,3 +159,8 @@ def test_binding_rejects_host_tensors():
     with pytest.raises(ValueError):
         ep.ep_layout(t, 1, 4, 2, 2, 1, t, t, t, t, torch.zeros(
             64, dtype=torch.uint8))
+    h = torch.zeros(4, 8, dtype=torch.bfloat16)
+    wt = torch.zeros(4, 2, dtype=torch.float32)
+    with pytest.raises(ValueError):
+        ep.ep_layout_dispatch(t, h, wt, 1, 4, 2, 2, 8, 1, False, t, t, t, t,
+                              h, workspace=torch.zeros(64, dtype=torch.uint8))
