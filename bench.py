@@ -476,6 +476,42 @@ def run_gpu(args, wl):
         avg[name] = replay_ms(g) / K * 1e3     # us per launch
         del g
     med = avg
+    # Per-call distribution: each call timed alone with CUDA events (eager
+    # launches, so the interval includes the launch), after writing a 512 MB
+    # scratch buffer (4x the L2) so that no call finds its inputs in L2; the
+    # small decode batch is also timed L2-hot, calls back to back.
+    per_call = {}
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    calls = {"layout_dispatch": path.layout_dispatch, "combine": path.combine}
+    if wl.B > 0:
+        calls["plan_prefetch"] = path.plan_prefetch
+    modes = [("l2_flushed", True)] + ([("l2_hot", False)]
+                                      if b_step < 512e6 else [])
+    for mode, do_flush in modes:
+        for name, fn in calls.items():
+            n_calls = 10 if name == "plan_prefetch" else 50
+            evs = []
+            if not do_flush:
+                # keep the GPU busy while the host enqueues the calls, so
+                # that they run back to back and each interval is GPU time
+                torch.cuda._sleep(4_000_000)
+            for _ in range(n_calls):
+                if do_flush:
+                    flush.fill_(1)
+                a_, b_ = (torch.cuda.Event(enable_timing=True),
+                          torch.cuda.Event(enable_timing=True))
+                a_.record()
+                fn()
+                b_.record()
+                evs.append((a_, b_))
+            torch.cuda.synchronize()
+            us = np.array([a_.elapsed_time(b_) * 1e3 for a_, b_ in evs])
+            per_call.setdefault(mode, {})[name] = {
+                "p10": round(float(np.percentile(us, 10)), 2),
+                "p50": round(float(np.percentile(us, 50)), 2),
+                "p90": round(float(np.percentile(us, 90)), 2),
+                "calls": n_calls}
+    del flush
     ms = start.elapsed_time(stop)
     ms_max = rank_max(ms)
     st = int(path.status[0].item())
@@ -544,6 +580,7 @@ def run_gpu(args, wl):
                           "once, CUDA events around the replay; per-kernel "
                           "times from a graph of K launches of that kernel",
             },
+            "per_call_us": per_call,
             "breakdown": {
                 "layout_dispatch_us": round(med["layout_dispatch"], 2),
                 "layout_dispatch_GBps": round(ld_gbs, 1),
@@ -729,6 +766,44 @@ def cpu_baseline(wl, n_tok):
                       "of the sample, single-threaded C"}
 
 
+def _oracle_worker(job):
+    """One process of the multi-core baseline: an independent synthetic
+    sample of the workload, timed after every process has built its inputs
+    (the barrier), on the wall clock shared by the processes."""
+    wl_name, scale_kw, n_tok, seed_offset, barrier = job
+    wl = workloads.WORKLOADS[wl_name]
+    if scale_kw:
+        wl = workloads.scaled(wl, **scale_kw)
+    topk, w, h, y = oracle_sample(wl, n_tok, seed_offset=seed_offset)
+    barrier.wait()
+    t0 = time.time()
+    dt, b = time_oracle_step(wl, topk, w, h, y)
+    return t0, t0 + dt, b
+
+
+def cpu_baseline_parallel(wl, n_tok, scale_kw):
+    """The same oracle step, unmodified, run by one process per available
+    core (capped at 32) on independent samples at once."""
+    import multiprocessing as mp
+    cores = len(os.sched_getaffinity(0))
+    procs = max(1, min(32, cores))
+    ctx = mp.get_context("spawn")   # the parent holds a CUDA context
+    with ctx.Manager() as mgr:
+        barrier = mgr.Barrier(procs)
+        with ctx.Pool(procs) as pool:
+            res = pool.map(_oracle_worker,
+                           [(wl.name, scale_kw, n_tok, 100 + i, barrier)
+                            for i in range(procs)])
+    t0 = min(r[0] for r in res)
+    t1 = max(r[1] for r in res)
+    b = sum(r[2] for r in res)
+    return {"value": round(b / (t1 - t0) / 1e9, 3), "unit": "GB/s",
+            "cores": procs, "kind": "oracle",
+            "seconds": round(t1 - t0, 2),
+            "sample": f"{procs} processes at once, each the single-threaded "
+                      f"oracle step on its own {n_tok}-token sample"}
+
+
 def run_reference(args, wl):
     ws, rank, _ = dist_info()
     if rank != 0:
@@ -800,6 +875,10 @@ def main():
         if ws == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(
                 wl, min(wl.N, args.cpu_sample_tokens))
+            scale_kw = ({"S": args.tokens_per_rank}
+                        if args.tokens_per_rank else None)
+            res["cpu_baseline_all_cores"] = cpu_baseline_parallel(
+                wl, min(wl.N, 1024), scale_kw)
         else:
             res["cpu_baseline"] = None
         print(json.dumps(res), flush=True)

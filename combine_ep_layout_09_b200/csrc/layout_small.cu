@@ -101,31 +101,43 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
 }
 
 
+// The count's loads: round i0 of the int4 loads over the top-k array
+// (topk is 16-byte aligned), kCountUnroll loads per thread per round.
+constexpr int kCountUnroll = 4;
+
+template <int NT>
+__device__ __forceinline__ void count_loads(const int32_t* __restrict__ topk,
+                                            int64_t M4, int64_t i0,
+                                            int4 (&v)[kCountUnroll]) {
+#pragma unroll
+  for (int u = 0; u < kCountUnroll; ++u) {
+    const int64_t i = i0 + int64_t(u) * NT * 4;
+    v[u] = i < M4 ? __ldg(reinterpret_cast<const int4*>(topk + i))
+                  : make_int4(-1, -1, -1, -1);
+  }
+}
+
 // Counts: every entry of the batch into before[e] (entries ahead of the
 // chunk) or after[e] (the chunk and later), and the chunk's own expert ids
-// into skey. Threads [0, NT).
+// into skey. Threads [0, NT). v holds the first round's loads, issued by the
+// caller before the shared memory was set up.
 template <int NT>
 __device__ __forceinline__ void count_entries(const int32_t* __restrict__ topk,
                                               int64_t M, int E, int64_t split,
                                               int n_ent, int32_t* before,
-                                              int32_t* after, int32_t* skey) {
+                                              int32_t* after, int32_t* skey,
+                                              int4 (&v)[kCountUnroll]) {
   auto count = [&](int e, int64_t i) {
     if (unsigned(e) < unsigned(E)) atomicAdd(i < split ? &before[e] : &after[e], 1);
     const int64_t r = i - split;
     if (r >= 0 && r < n_ent) skey[r] = e;
   };
-  const int64_t M4 = M & ~int64_t(3);  // topk is 16-byte aligned
-  constexpr int kU = 4;
-  for (int64_t i0 = int64_t(threadIdx.x) * 4; i0 < M4; i0 += int64_t(NT) * 4 * kU) {
-    int4 v[kU];
+  const int64_t M4 = M & ~int64_t(3);
+  for (int64_t i0 = int64_t(threadIdx.x) * 4; i0 < M4;
+       i0 += int64_t(NT) * 4 * kCountUnroll) {
+    if (i0 != int64_t(threadIdx.x) * 4) count_loads<NT>(topk, M4, i0, v);
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int64_t i = i0 + int64_t(u) * NT * 4;
-      v[u] = i < M4 ? __ldg(reinterpret_cast<const int4*>(topk + i))
-                    : make_int4(-1, -1, -1, -1);
-    }
-#pragma unroll
-    for (int u = 0; u < kU; ++u) {
+    for (int u = 0; u < kCountUnroll; ++u) {
       const int64_t i = i0 + int64_t(u) * NT * 4;
       if (i < M4) {
         count(v[u].x, i);
@@ -308,6 +320,9 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
              &full[s]);
   };
 
+  // the count's first loads go out before the shared-memory setup
+  int4 v0[kCountUnroll];
+  count_loads<kSmallThreads>(topk, (N * K) & ~int64_t(3), int64_t(tid) * 4, v0);
   if (tid == 0) {
     s_abort = 0;
     s_next = 0;
@@ -340,7 +355,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
       const int j = tid + q * kSmallThreads;
       wv[q] = (want_w && j < n_ent) ? __ldg(w + split + j) : 0.0f;
     }
-    count_entries<kSmallThreads>(topk, N * K, E, split, n_ent, before, after, skey);
+    count_entries<kSmallThreads>(topk, N * K, E, split, n_ent, before, after, skey, v0);
 #pragma unroll
     for (int q = 0; q < kPerThread; ++q) {
       const int j = tid + q * kSmallThreads;
