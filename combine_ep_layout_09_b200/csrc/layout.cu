@@ -21,10 +21,12 @@
 // a hardware match whose cost grows with the number of distinct keys.
 //
 // Two paths here (small batches, N*K <= 32768, take layout_small.cu instead):
-//   fused      (tiles fit co-resident) one cooperative launch: the last tile's
-//              inclusive prefix holds every expert's total; every tile reads
-//              it, scans the padded totals into the expert offsets itself,
-//              and writes final positions from the ranks kept in registers.
+//   fused      (tiles fit co-resident) one cooperative launch: every tile
+//              publishes its per-expert counts once; once all have, each
+//              tile sums them (reduce-then-scan: the counts of the tiles
+//              before it, and the totals), scans the padded totals into the
+//              expert offsets itself, and writes final positions from the
+//              ranks kept in registers. No look-back chain.
 //   two-kernel (any size) k_histogram counts with warp-aggregated shared-memory
 //              atomics and its last CTA writes the offsets; k_scan_positions
 //              then ranks, looks back and writes positions, tile ids claimed
@@ -283,7 +285,8 @@ __device__ __forceinline__ bool rank_in_warps(const int32_t* __restrict__ topk,
 __device__ __forceinline__ void tile_totals_publish(int32_t* whist,
                                                     int32_t* tcount,
                                                     int32_t* part, int E,
-                                                    int tile, uint32_t* desc) {
+                                                    int tile, uint32_t* desc,
+                                                    bool first_inclusive = true) {
   const int tpe = max(1, min(kScanWarps, kScanThreads / E));  // threads / expert
   const int chunk = (kScanWarps + tpe - 1) / tpe;             // warps / thread
   for (int j = threadIdx.x; j < E * tpe; j += kScanThreads) {
@@ -306,7 +309,8 @@ __device__ __forceinline__ void tile_totals_publish(int32_t* whist,
     }
     tcount[e] = run;
     st_relaxed_gpu(desc + int64_t(tile) * E + e,
-                   (tile == 0 ? kFlagInclusive : kFlagAggregate) | uint32_t(run));
+                   (tile == 0 && first_inclusive ? kFlagInclusive : kFlagAggregate) |
+                       uint32_t(run));
   }
   __syncthreads();
   for (int j = threadIdx.x; j < E * tpe; j += kScanThreads) {
@@ -336,6 +340,72 @@ __device__ __forceinline__ void tile_lookback(const int32_t* tcount,
     }
   }
   __syncthreads();  // excl[e] was written by thread 2e, not by thread e
+}
+
+// Fused path: every tile's counts are published once (never overwritten),
+// so each tile reads them all once every tile has published: excl[e] =
+// entries of e in the tiles before this one, tot[e] = in all tiles. P
+// threads share an expert, each summing tiles j = p, p+P, ... with
+// kReduceBatch loads in flight; the P partial sums meet in `scratch`
+// ([2][P][E] ints).
+constexpr int kReduceBatch = 16;
+__device__ __forceinline__ void tile_reduce(const uint32_t* desc, int E, int tile,
+                                            int num_tiles, int32_t* excl,
+                                            int32_t* tot, int32_t* scratch,
+                                            int32_t* status) {
+  const int P = max(1, min(32, kScanThreads / E));
+  for (int idx = threadIdx.x; idx < E * P; idx += kScanThreads) {
+    const int e = idx % E, p = idx / E;
+    uint32_t sx = 0, st = 0;
+    for (int j0 = p; j0 < num_tiles; j0 += P * kReduceBatch) {
+      uint32_t v[kReduceBatch];
+      unsigned pending = 0;
+#pragma unroll
+      for (int q = 0; q < kReduceBatch; ++q) {
+        const int j = j0 + q * P;
+        v[q] = kFlagAggregate;
+        if (j < num_tiles) {
+          v[q] = ld_relaxed_gpu(desc + int64_t(j) * E + e);
+          if ((v[q] & ~kValueMask) == 0u) pending |= 1u << q;
+        }
+      }
+      if (pending) {  // some tile has not published yet: poll those
+        const uint64_t t0 = globaltimer_ns();
+        while (pending) {
+#pragma unroll
+          for (int q = 0; q < kReduceBatch; ++q)
+            if ((pending >> q) & 1u) {
+              v[q] = ld_relaxed_gpu(desc + int64_t(j0 + q * P) * E + e);
+              if ((v[q] & ~kValueMask) != 0u) pending &= ~(1u << q);
+            }
+          if (pending && globaltimer_ns() - t0 > kWaitBudgetNs) {
+            report(status, EP_DEV_TIMEOUT);
+            break;
+          }
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < kReduceBatch; ++q) {
+        const int j = j0 + q * P;
+        const uint32_t c = v[q] & kValueMask;
+        st += c;
+        if (j < tile) sx += c;
+      }
+    }
+    scratch[p * E + e] = int32_t(sx);
+    scratch[(P + p) * E + e] = int32_t(st);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kScanThreads) {
+    int32_t a = 0, b = 0;
+    for (int p = 0; p < P; ++p) {
+      a += scratch[p * E + e];
+      b += scratch[(P + p) * E + e];
+    }
+    excl[e] = a;
+    tot[e] = b;
+  }
+  __syncthreads();
 }
 
 // pos and row_src of the tile's entries. base[e] = first row of expert e
@@ -477,7 +547,6 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   __shared__ int32_t s_warp2[2 * kScanThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int tile = blockIdx.x;
-  const bool last = (tile == num_tiles - 1);
 
   for (int j = tid; j < kScanWarps * E; j += kScanThreads) sm.whist[j] = 0;
   __syncthreads();
@@ -487,33 +556,13 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   const bool bad = rank_in_warps(topk, M, E, wbase, my, kr);
   if (__any_sync(0xffffffffu, bad) && lane == 0) report(status, EP_DEV_BAD_EXPERT);
   __syncthreads();
-  tile_totals_publish(sm.whist, sm.tcnt, sm.part, E, tile, desc);
-  tile_lookback(sm.tcnt, sm.base, E, tile, desc, status);
-
-  // Every expert's total is the last tile's inclusive prefix: the last tile
-  // has it now, the others read its descriptors (every CTA of a cooperative
-  // launch is resident, so the last tile will publish). Then each tile scans
-  // the padded totals into expert offsets and its own counts into its
-  // counting-sort prefix, in one pass.
+  // counts published as aggregates only; every tile then reads all of them
+  tile_totals_publish(sm.whist, sm.tcnt, sm.part, E, tile, desc, false);
+  tile_reduce(desc, E, tile, num_tiles, sm.base, sm.tot, sm.sorted, status);
+  // each tile scans the padded totals into expert offsets and its own counts
+  // into its counting-sort prefix, in one pass
   for (int e = tid; e < E; e += kScanThreads) {
-    int32_t total;
-    if (last) {
-      total = sm.base[e] + sm.tcnt[e];
-    } else {
-      const uint32_t* d = desc + int64_t(num_tiles - 1) * E + e;
-      uint32_t v = ld_relaxed_gpu(d);
-      if ((v & ~kValueMask) != kFlagInclusive) {
-        const uint64_t t0 = globaltimer_ns();
-        while (((v = ld_relaxed_gpu(d)) & ~kValueMask) != kFlagInclusive) {
-          if (globaltimer_ns() - t0 > kWaitBudgetNs) {
-            report(status, EP_DEV_TIMEOUT);
-            break;
-          }
-        }
-      }
-      total = int32_t(v & kValueMask);
-    }
-    sm.tot[e] = total;
+    const int32_t total = sm.tot[e];
     sm.offs[e] = int32_t(((int64_t(total) + pad - 1) / pad) * pad);
     sm.tpre[e] = sm.tcnt[e];
   }
@@ -524,7 +573,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     sm.offs[E] = rows_used;
     sm.tpre[E] = tile_n;
   }
-  if (last) {
+  if (tile == num_tiles - 1) {
     for (int e = tid; e < E; e += kScanThreads) {
       tokens_per_expert[e] = sm.tot[e];
       expert_offsets[e] = sm.offs[e];

@@ -105,7 +105,8 @@ EP_API size_t ep_layout_workspace_bytes(int64_t num_tokens, int K, int E);
  * Launches on `stream`: for N*K <= 32768 (and at most 1024 entries per
  * SM) one kernel in which every CTA counts all entries and places its own
  * tokens, workspace unused; above that a memset and one cooperative kernel
- * (a decoupled look-back scan), or a memset and two kernels when the tiles
+ * (tiles that sum each other's published counts), or a memset and two
+ * kernels (a histogram, then a decoupled look-back scan) when the tiles
  * cannot all be resident.
  */
 EP_API int ep_layout(const int32_t* topk_experts, int R, int S, int K, int E,
