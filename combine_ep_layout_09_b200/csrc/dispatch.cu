@@ -9,9 +9,9 @@
 // kernels), with no later permutation.
 //
 // Both kernels move rows with the TMA engine's 1-D bulk copies (no tensor
-// map, no multicast): a token row comes into shared memory once and leaves
-// K times. The kernel reads 1/(K+1) of the bytes it moves, so HBM write
-// bandwidth bounds it.
+// map; each CTA loads only its own rows): a token row comes into shared
+// memory once and leaves K times. The kernel reads 1/(K+1) of the bytes it
+// moves, so HBM write bandwidth bounds it.
 //
 //   k_dispatch_bf16  one-warp CTAs; lane 0 keeps a ring of token rows in
 //                    flight and, per row, issues K bulk stores from shared
