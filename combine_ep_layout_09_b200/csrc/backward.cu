@@ -116,14 +116,16 @@ __global__ void __launch_bounds__(kBwdMaxThreads)
   const int64_t gw = int64_t(blockIdx.x) * nwarps + warp;
   const int64_t gstride = int64_t(gridDim.x) * nwarps;
   const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-  for (int64_t r0 = gw * 32; r0 < used; r0 += gstride * 32) {
-    const int64_t r = r0 + lane;
+  // lane l of warp gw looks at row gw + (32*i + l) * gstride, so that the
+  // padding rows of one expert (a contiguous run) fall to different warps
+  for (int64_t i0 = 0; gw + i0 * gstride < used; i0 += 32) {
+    const int64_t r = gw + (i0 + lane) * gstride;
     const bool is_pad = r < used && __ldg(row_src + r) < 0;
     unsigned m = __ballot_sync(0xffffffffu, is_pad);
     while (m) {
       const int bit = __ffs(m) - 1;
       m &= m - 1;
-      const int64_t row = r0 + bit;
+      const int64_t row = gw + (i0 + bit) * gstride;
       for (int v = lane; v < V; v += 32) st_v4(grad_rows + row * H + v * 8, z);
     }
   }

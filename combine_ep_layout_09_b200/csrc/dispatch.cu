@@ -61,14 +61,16 @@ __device__ void zero_padding_rows(const int32_t* __restrict__ row_src,
   const int64_t gstride = int64_t(gridDim.x) * nwarps;
   const int G = H >> 7;
   const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-  for (int64_t r0 = gw * 32; r0 < used; r0 += gstride * 32) {
-    const int64_t r = r0 + lane;
+  // Lane l of warp gw looks at row gw + (32*i + l) * gstride: the padding
+  // rows of one expert (a contiguous run) fall to different warps.
+  for (int64_t i0 = 0; gw + i0 * gstride < used; i0 += 32) {
+    const int64_t r = gw + (i0 + lane) * gstride;
     const bool is_pad = r < used && __ldg(row_src + r) < 0;
     unsigned m = __ballot_sync(0xffffffffu, is_pad);
     while (m) {
       const int bit = __ffs(m) - 1;
       m &= m - 1;
-      const int64_t row = r0 + bit;
+      const int64_t row = gw + (i0 + bit) * gstride;
       if constexpr (kFp8) {
         for (int c = lane * 16; c < H; c += 32 * 16) st_v4(recv + row * H + c, z);
         for (int g = lane; g < G; g += 32) scales[row * G + g] = 0.0f;
