@@ -320,17 +320,38 @@ __global__ void __launch_bounds__(kRedThreads)
     const int e = s_exp[j0];
     float4* G = proj == 0 ? g0 : (proj == 1 ? g1 : g2);
     const int64_t lo = ch * kRedVec, hi = min(vecs, lo + kRedVec);
-    for (int64_t v = lo + tid; v < hi; v += kRedThreads) {
-      float4 acc = G[int64_t(e) * vecs + v];
+    // four vectors per thread per round: their loads go out together
+    for (int64_t vb = lo + tid; vb < hi; vb += 4 * kRedThreads) {
+      float4 acc[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int64_t v = vb + int64_t(q) * kRedThreads;
+        if (v < hi) acc[q] = G[int64_t(e) * vecs + v];
+      }
       for (int j = j0; j < n; ++j) {
         if (s_exp[j] != e) continue;
-        const float4 x = G[(int64_t(E) + s_slot[j]) * vecs + v];
-        acc.x = acc.x + x.x;
-        acc.y = acc.y + x.y;
-        acc.z = acc.z + x.z;
-        acc.w = acc.w + x.w;
+        float4 x[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int64_t v = vb + int64_t(q) * kRedThreads;
+          if (v < hi) x[q] = G[(int64_t(E) + s_slot[j]) * vecs + v];
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int64_t v = vb + int64_t(q) * kRedThreads;
+          if (v < hi) {
+            acc[q].x = acc[q].x + x[q].x;
+            acc[q].y = acc[q].y + x[q].y;
+            acc[q].z = acc[q].z + x[q].z;
+            acc[q].w = acc[q].w + x[q].w;
+          }
+        }
       }
-      G[int64_t(e) * vecs + v] = acc;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int64_t v = vb + int64_t(q) * kRedThreads;
+        if (v < hi) G[int64_t(e) * vecs + v] = acc[q];
+      }
     }
   }
 }
@@ -423,7 +444,7 @@ cudaError_t launch_reduce_slot_grads(const int32_t* slot_expert, int R, int E,
   const int64_t vecs = elems / 4;
   const int64_t nchunk = (vecs + kRedVec - 1) / kRedVec;
   const int64_t grid = std::max<int64_t>(
-      1, std::min<int64_t>(RB * 3 * nchunk, int64_t(num_sms) * 4));
+      1, std::min<int64_t>(RB * 3 * nchunk, int64_t(num_sms) * 8));
   k_reduce_slot_grads<<<int(grid), kRedThreads, 0, stream>>>(
       slot_expert, int(RB), E, vecs, reinterpret_cast<float4*>(g0),
       reinterpret_cast<float4*>(g1), reinterpret_cast<float4*>(g2));
