@@ -82,3 +82,28 @@ def test_plan_prefetch_reduce_and_backward_through_the_buffer():
     torch.cuda.synchronize()
     a, b = gx.float(), grad_out.float()
     assert bool(((a - b).abs() <= b.abs() * 2.0 ** -7 + 1e-30).all())
+
+
+def test_double_buffer_on_the_large_batch_kernels():
+    # 4800 tokens x top-8: layout and dispatch are two kernels, the dispatch a
+    # programmatic dependent of the layout; two batches in flight on the two
+    # receive sets, each checked against the oracle afterwards
+    wl = workloads.scaled(workloads.WORKLOADS["prefill"], S=600, H=512)
+    topk, w = workloads.routing(wl)
+    topk2 = np.roll(topk, 7, axis=0)
+    buf = EPBuffer(wl.S, wl.H, wl.K, wl.E, wl.R, fp8=True, double_buffer=True)
+    h1 = workloads.hidden_states(wl, device=DEV)
+    h2 = workloads.bf16_normal((wl.N, wl.H), 77, device=DEV)
+    r1, rw1, _, hd1 = buf.dispatch(h1, to_dev(w), to_dev(topk))
+    r2, rw2, _, hd2 = buf.dispatch(h2, to_dev(w), to_dev(topk2))
+    torch.cuda.synchronize()
+    buf.check()
+    for hid, tk, r, hd in ((h1, topk, r1, hd1), (h2, topk2, r2, hd2)):
+        lay = oracle.layout(tk, wl.E, wl.pad, buf.cap)
+        used = int(lay["offsets"][-1])
+        np.testing.assert_array_equal(hd.pos.cpu().numpy(), lay["pos"])
+        q, s, _ = oracle.dispatch_fp8(u16(hid), w, lay, wl.E, buf.cap)
+        np.testing.assert_array_equal(r.view(torch.uint8).cpu().numpy()[:used],
+                                      q[:used])
+        np.testing.assert_array_equal(hd.recv_scales.cpu().numpy()[:used],
+                                      s[:used])
