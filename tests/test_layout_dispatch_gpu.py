@@ -176,3 +176,12 @@ def test_duplicate_ids_single_expert_and_wide_padding(fp8):
     check(topk, w, h, R, S, E, 1, fp8)
     check(np.full((R * S, K), 1, np.int32), w, h, R, S, E, 7, fp8)
     check(topk, w, h, R, S, E, 1000, fp8)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_small_batch_on_one_sm_takes_two_launches(fp8):
+    # 256 tokens x 8 on one SM would put 2048 entries on one CTA, above its
+    # limit of 1024: the call runs the layout and dispatch kernels instead
+    R, S, K, E, H = 2, 128, 8, 32, 1024
+    topk, w, h = make(23, R * S, K, E, H, distinct=True)
+    check(topk, w, h, R, S, E, 2, fp8, num_sms=1)
