@@ -1,0 +1,61 @@
+"""bench.py's byte accounting against the figures it is defined by, and its
+launch count against the library's size rule (host only)."""
+import os
+import re
+
+import pytest
+
+import bench
+import workloads
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_prefill_and_decode_bytes():
+    # each input read once, each output written once: hidden 2 B/channel,
+    # FP8 codes 1 B/channel + one fp32 scale per 128 channels + a weight per
+    # row; combine reads K bf16 rows and writes one
+    N, K, H = 32768, 8, 7168
+    rows = N * K
+    disp = bench.bytes_dispatch(N, K, H, True, rows)
+    assert disp == (N * H * 2 + N * K * 8 + rows * 4 +
+                    rows * (H + H // 128 * 4 + 4))
+    assert abs(disp / 1e6 - 2411.7) < 0.1
+    assert abs(bench.bytes_combine(N, K, H) / 1e6 - 4230.0) < 0.1
+    dec = workloads.WORKLOADS["decode"]
+    d = bench.bytes_dispatch(dec.N, dec.K, dec.H, True, dec.N * dec.K)
+    assert abs(d / 1e6 - 75.37) < 0.01
+    # bf16 rows are twice as wide; padding rows count as written rows
+    assert (bench.bytes_dispatch(N, K, H, False, rows + 100) -
+            bench.bytes_dispatch(N, K, H, False, rows)) == 100 * (2 * H + 4) + 100 * 4
+
+
+def test_reduce_bytes_per_slot_group():
+    import numpy as np
+    slots = np.array([[3, -1], [3, 7]], np.int32)   # expert 3 twice, 7 once
+    H, I = 8, 4
+    # expert 3: own row read + written, 2 slot rows read; expert 7: 1 slot
+    assert bench.bytes_reduce_slot_grads(slots, H, I) == 3 * (4 + 3) * H * I * 4
+
+
+def _header_constant(name):
+    src = open(os.path.join(ROOT, "combine_ep_layout_09_b200", "csrc",
+                            "ep_launch.h")).read()
+    m = re.search(r"constexpr\s+int64_t\s+%s\s*=\s*(\d+)\s*;" % name, src)
+    assert m, name
+    return int(m.group(1))
+
+
+@pytest.mark.parametrize("S,K,expect", [
+    (128, 8, 1),      # decode: 8192 entries, 7 tokens per CTA
+    (512, 8, 1),      # 32768 entries exactly
+    (513, 8, 2),      # one tile more: cooperative layout + dispatch
+    (4096, 8, 2),     # prefill: 64 tiles, all resident
+    (49152, 8, 3),    # 768 tiles: histogram + scan + dispatch
+])
+def test_launch_count_follows_the_library_rule(S, K, expect):
+    limit = _header_constant("kSmallMaxEntries")
+    per_cta = _header_constant("kSmallMaxChunkEntries")
+    assert (limit, per_cta) == (32768, 1024)   # the numbers bench.py mirrors
+    wl = workloads.scaled(workloads.WORKLOADS["prefill"], S=S, K=K)
+    assert bench.layout_dispatch_kernels(wl) == expect
