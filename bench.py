@@ -339,7 +339,8 @@ class Path:
         self.ep.ep_plan_balanced(self.counts, wl.R, wl.S, wl.K, wl.E, wl.B,
                                  p["cu"], p["expert"], p["wrow"], p["nseg"],
                                  p["slot"], self.status)
-        self.ep.ep_prefetch_weights(p["slot"], wl.R, wl.E, wl.B, *self.W)
+        self.ep.ep_prefetch_weights(p["slot"], wl.R, wl.E, wl.B, *self.W,
+                                    status=self.status)
 
     def layout_dispatch(self, io=None):
         """The user's dispatch call: layout and copy (one launch for a small

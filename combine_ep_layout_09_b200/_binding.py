@@ -30,6 +30,14 @@ EP_DEV_TIMEOUT = 4
 EP_DEV_SLOTS = 8
 EP_DEV_PLAN_TOTAL = 16
 
+EP_WAIT_SITE_LOOKBACK = 1
+EP_WAIT_SITE_TILE_REDUCE = 2
+EP_WAIT_SITE_DISPATCH = 4
+EP_WAIT_SITE_COMBINE = 8
+EP_WAIT_SITE_SMALL = 16
+EP_WAIT_SITE_PREFETCH = 32
+EP_WAIT_SITE_ALL = 63
+
 _lock = threading.Lock()
 _lib = None
 
@@ -87,6 +95,9 @@ def _declare(L):
                                      i32, P, P]
     L.ep_combine.restype = i32
     L.ep_combine.argtypes = [P, P, P, i64, i32, i32, i64, P, i32, P, P]
+    L.ep_combine_recv_weights.restype = i32
+    L.ep_combine_recv_weights.argtypes = [P, P, P, i64, i32, i32, i64, P, P,
+                                          i32, P, P]
     L.ep_dispatch_backward.restype = i32
     L.ep_dispatch_backward.argtypes = [P, P, i64, i32, i32, i64, P, i32, P, P]
     L.ep_combine_backward.restype = i32
@@ -98,7 +109,8 @@ def _declare(L):
     L.ep_plan_balanced.argtypes = [P, i32, i32, i32, i32, i32, P, P, P, P, P,
                                    P, P]
     L.ep_prefetch_weights.restype = i32
-    L.ep_prefetch_weights.argtypes = [P, i32, i32, i32, i64, P, P, P, i32, P]
+    L.ep_prefetch_weights.argtypes = [P, i32, i32, i32, i64, P, P, P, i32, P,
+                                      P]
     L.ep_reduce_slot_grads.restype = i32
     L.ep_reduce_slot_grads.argtypes = [P, i32, i32, i32, i64, P, P, P, i32, P]
     L.ep_debug_e4m3_encode.restype = i32
@@ -107,6 +119,8 @@ def _declare(L):
     L.ep_debug_quantize.argtypes = [P, P, P, i64, P]
     L.ep_debug_bounded_wait.restype = i32
     L.ep_debug_bounded_wait.argtypes = [P, i64, P, P]
+    L.ep_debug_force_timeouts.restype = i32
+    L.ep_debug_force_timeouts.argtypes = [ctypes.c_uint32, i64]
 
 
 # --------------------------------------------------------------------------
@@ -266,6 +280,25 @@ def ep_combine(expert_out, pos, route_weights, num_tokens, K, H, out,
     _check(rc, "ep_combine")
 
 
+def ep_combine_recv_weights(expert_out, pos, recv_weights, num_tokens, K, H,
+                            out, gathered=None, num_sms=0, status=None,
+                            cap=None, stream=None):
+    """Combine with the receive-side weights recv_weights[pos[t,k]]; the
+    weights also come back in token order in `gathered` (may be None)."""
+    cap = expert_out.shape[0] if cap is None else int(cap)
+    rc = lib().ep_combine_recv_weights(
+        _ptr(expert_out, "expert_out", _BF16, cap * H),
+        _ptr(pos, "pos", _I32, num_tokens * K),
+        _ptr(recv_weights, "recv_weights", _F32, cap),
+        num_tokens, K, H, cap,
+        _ptr(out, "out", _BF16, num_tokens * H),
+        _ptr(gathered, "gathered", _F32, num_tokens * K, optional=True),
+        int(num_sms),
+        _ptr(status, "status", _I32, 1, optional=True),
+        _stream(stream))
+    _check(rc, "ep_combine_recv_weights")
+
+
 def ep_dispatch_backward(grad_recv, pos, num_tokens, K, H, grad_hidden,
                          num_sms=0, status=None, cap=None, stream=None):
     """grad_hidden[t] = bf16(sum_k grad_recv[pos[t,k]]) in fp32, k order."""
@@ -329,7 +362,7 @@ def ep_plan_balanced(tokens_per_expert, R, S, K, E, B, plan_cu, plan_expert,
 
 
 def ep_prefetch_weights(slot_expert, R, E, B, gate, up, down, num_sms=0,
-                        stream=None):
+                        status=None, stream=None):
     """Copy the slot experts' gate/up/down rows into the prefetch slots."""
     rows = E + R * B
     elems = gate[0].numel() if gate.shape[0] > 0 else 0
@@ -341,7 +374,8 @@ def ep_prefetch_weights(slot_expert, R, E, B, gate, up, down, num_sms=0,
         R, E, B, elems,
         _ptr(gate, "gate", _W16), _ptr(up, "up", _W16),
         _ptr(down, "down", _W16),
-        int(num_sms), _stream(stream))
+        int(num_sms), _ptr(status, "status", _I32, 1, optional=True),
+        _stream(stream))
     _check(rc, "ep_prefetch_weights")
 
 
@@ -382,3 +416,10 @@ def ep_debug_bounded_wait(flag, max_polls, status, stream=None):
         _ptr(flag, "flag", _I32, 1), int(max_polls),
         _ptr(status, "status", _I32, 1), _stream(stream))
     _check(rc, "ep_debug_bounded_wait")
+
+
+def ep_debug_force_timeouts(sites, budget_ns=0):
+    """Make the waits at `sites` (EP_WAIT_SITE_* bits) give up after
+    budget_ns on the current device; sites=0 restores normal waits."""
+    rc = lib().ep_debug_force_timeouts(int(sites), int(budget_ns))
+    _check(rc, "ep_debug_force_timeouts")

@@ -62,6 +62,10 @@ class _Set:
             self.recv = torch.empty(rows, H, dtype=torch.bfloat16, device=dev)
             self.recv_scales = None
         self.recv_weights = torch.empty(rows, dtype=torch.float32, device=dev)
+        # combine's outputs, reused by every combine on this set
+        self.out = torch.empty(max(N, 1), H, dtype=torch.bfloat16, device=dev)
+        self.gathered = torch.empty(max(N, 1), K, dtype=torch.float32,
+                                    device=dev)
 
 
 class EPBuffer:
@@ -144,7 +148,8 @@ class EPBuffer:
                         full_down_weight, stream=None):
         B.ep_prefetch_weights(plan["slot_expert"], self.R, self.E, plan["B"],
                               full_gate_weight, full_up_weight,
-                              full_down_weight, self.num_sms, stream=stream)
+                              full_down_weight, self.num_sms, self.status,
+                              stream=stream)
 
     def reduce_grads(self, plan: dict, grad_gate, grad_up, grad_down,
                      stream=None):
@@ -156,24 +161,28 @@ class EPBuffer:
     # -- combine ---------------------------------------------------------------
     def combine(self, handle: DispatchHandle, expert_output: torch.Tensor,
                 route_weights_nvs: torch.Tensor | None = None,
-                out: torch.Tensor | None = None, stream=None):
-        """-> (output_sh, gathered_route_weights_sk). The weights used are the
-        receive-side route_weights_nvs gathered back into token order (the
-        dispatch's recv_weights when None)."""
+                out: torch.Tensor | None = None,
+                gathered: torch.Tensor | None = None, stream=None):
+        """-> (output_sh, gathered_route_weights_sk). Each entry's weight is
+        the receive-side route_weights_nvs at its row (the dispatch's
+        recv_weights when None); one launch computes the output and hands
+        the weights back in token order. Unless `out` / `gathered` are
+        given, the results are the handle's buffer set's own tensors,
+        allocated at construction and overwritten by the next combine on
+        that set."""
+        st = self.sets[handle.index]
         rw = handle.recv_weights if route_weights_nvs is None else \
             route_weights_nvs
-        gathered = torch.empty(self.N, self.K, dtype=torch.float32,
-                               device=expert_output.device)
-        B.ep_gather_route_weights(rw, handle.pos, self.N, self.K, gathered,
-                                  cap=rw.numel(), stream=stream)
-        if out is None:
-            out = torch.empty(self.N, self.H, dtype=torch.bfloat16,
-                              device=expert_output.device)
-        # rows of expert_output bound the positions it may be read at
-        B.ep_combine(expert_output, handle.pos, gathered, self.N, self.K,
-                     self.H, out, self.num_sms, self.status,
-                     cap=expert_output.shape[0], stream=stream)
-        return out, gathered
+        out = st.out if out is None else out
+        gathered = st.gathered if gathered is None else gathered
+        # rows of expert_output (and of the weights) bound the positions
+        # that may be read
+        B.ep_combine_recv_weights(expert_output, handle.pos, rw, self.N,
+                                  self.K, self.H, out, gathered,
+                                  self.num_sms, self.status,
+                                  cap=min(expert_output.shape[0], rw.numel()),
+                                  stream=stream)
+        return out[:self.N], gathered[:self.N]
 
     # -- backward --------------------------------------------------------------
     def combine_backward(self, handle: DispatchHandle, grad_out, expert_output,

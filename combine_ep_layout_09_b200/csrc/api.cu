@@ -8,7 +8,7 @@
 
 namespace {
 
-constexpr int kAbiVersion = 3;
+constexpr int kAbiVersion = 4;  // 4: ep_combine_recv_weights, ep_debug_force_timeouts, prefetch status
 constexpr int kMaxK = 32;
 constexpr int kMaxH = 32768;
 constexpr int64_t kMaxEntries = (int64_t(1) << 30) - 1;
@@ -197,9 +197,32 @@ int ep_combine(const void* expert_out, const int32_t* pos,
   if (!aligned16(pos) || !aligned16(route_weights) || !aligned16(out))
     return EP_ERR_ALIGNMENT;
   if (cap > 0 && !aligned16(expert_out)) return EP_ERR_ALIGNMENT;
-  return cuda_rc(ep::launch_combine(expert_out, pos, route_weights, num_tokens,
-                                    K, H, cap, out, sms_or_all(num_sms),
-                                    status, as_stream(stream)));
+  return cuda_rc(ep::launch_combine(expert_out, pos, route_weights, nullptr,
+                                    nullptr, num_tokens, K, H, cap, out,
+                                    sms_or_all(num_sms), status,
+                                    as_stream(stream)));
+}
+
+int ep_combine_recv_weights(const void* expert_out, const int32_t* pos,
+                            const float* recv_weights, int64_t num_tokens,
+                            int K, int H, int64_t cap, void* out,
+                            float* gathered_route_weights, int num_sms,
+                            int32_t* status, void* stream) {
+  if (num_tokens < 0 || K < 1 || K > kMaxK || H < 8 || H > kMaxH ||
+      H % 8 != 0 || cap < 0 || cap > INT32_MAX || num_sms < 0 ||
+      num_tokens * K > kMaxEntries)
+    return EP_ERR_INVALID_ARG;
+  if (!status_ok(status)) return EP_ERR_ALIGNMENT;
+  if (num_tokens == 0) return EP_OK;
+  if (!aligned16(pos) || !aligned16(out) || !aligned16(recv_weights))
+    return EP_ERR_ALIGNMENT;
+  if (gathered_route_weights && !aligned16(gathered_route_weights))
+    return EP_ERR_ALIGNMENT;
+  if (cap > 0 && !aligned16(expert_out)) return EP_ERR_ALIGNMENT;
+  return cuda_rc(ep::launch_combine(expert_out, pos, nullptr, recv_weights,
+                                    gathered_route_weights, num_tokens, K, H,
+                                    cap, out, sms_or_all(num_sms), status,
+                                    as_stream(stream)));
 }
 
 int ep_dispatch_backward(const void* grad_recv, const int32_t* pos,
@@ -214,9 +237,10 @@ int ep_dispatch_backward(const void* grad_recv, const int32_t* pos,
   if (num_tokens == 0) return EP_OK;
   if (!aligned16(pos) || !aligned16(grad_hidden)) return EP_ERR_ALIGNMENT;
   if (cap > 0 && !aligned16(grad_recv)) return EP_ERR_ALIGNMENT;
-  return cuda_rc(ep::launch_combine(grad_recv, pos, nullptr, num_tokens, K, H,
-                                    cap, grad_hidden, sms_or_all(num_sms),
-                                    status, as_stream(stream)));
+  return cuda_rc(ep::launch_combine(grad_recv, pos, nullptr, nullptr, nullptr,
+                                    num_tokens, K, H, cap, grad_hidden,
+                                    sms_or_all(num_sms), status,
+                                    as_stream(stream)));
 }
 
 int ep_combine_backward(const void* grad_out, const void* expert_out,
@@ -278,17 +302,19 @@ int ep_plan_balanced(const int32_t* tokens_per_expert, int R, int S, int K,
 
 int ep_prefetch_weights(const int32_t* slot_expert, int R, int E, int B,
                         int64_t elems_per_expert, void* gate, void* up,
-                        void* down, int num_sms, void* stream) {
+                        void* down, int num_sms, int32_t* status,
+                        void* stream) {
   if (R < 1 || E < 1 || B < 0 || elems_per_expert < 0 ||
       (elems_per_expert * 2) % 16 != 0 || num_sms < 0)
     return EP_ERR_INVALID_ARG;
+  if (!status_ok(status)) return EP_ERR_ALIGNMENT;
   if (B == 0 || elems_per_expert == 0) return EP_OK;
   if (!aligned16(slot_expert) || !aligned16(gate) || !aligned16(up) ||
       !aligned16(down))
     return EP_ERR_ALIGNMENT;
   return cuda_rc(ep::launch_prefetch(slot_expert, R, E, B, elems_per_expert,
                                      gate, up, down, sms_or_all(num_sms),
-                                     as_stream(stream)));
+                                     status, as_stream(stream)));
 }
 
 int ep_reduce_slot_grads(const int32_t* slot_expert, int R, int E, int B,
@@ -333,6 +359,20 @@ int ep_debug_bounded_wait(const int32_t* flag, int64_t max_polls,
   if (!aligned16(flag) || status == nullptr || !status_ok(status))
     return EP_ERR_ALIGNMENT;
   return cuda_rc(ep::launch_debug_wait(flag, max_polls, status, as_stream(stream)));
+}
+
+int ep_debug_force_timeouts(uint32_t sites, int64_t budget_ns) {
+  if ((sites & ~uint32_t(EP_WAIT_SITE_ALL)) != 0u ||
+      (sites != 0u && (budget_ns <= 0 || budget_ns > 2000000000)))
+    return EP_ERR_INVALID_ARG;
+  const uint64_t b = uint64_t(budget_ns);
+  cudaError_t (*const setters[])(uint32_t, uint64_t) = {
+      ep::set_wait_debug_layout, ep::set_wait_debug_layout_small,
+      ep::set_wait_debug_dispatch, ep::set_wait_debug_combine,
+      ep::set_wait_debug_plan};
+  for (auto set : setters)
+    if (set(sites, b) != cudaSuccess) return EP_ERR_CUDA;
+  return EP_OK;
 }
 
 }  // extern "C"

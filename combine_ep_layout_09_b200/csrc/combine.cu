@@ -18,6 +18,13 @@
 //                  into 16-byte vectors and issue their K gathered loads
 //                  before any arithmetic.
 // Both run the same fma chain in the same k order.
+//
+// Weights come either per entry (w[t,k], token side) or per receive row
+// (w_rows[pos[t,k]]: the receive-side route_weights_nvs of
+// "MoonEP核心功能深度剖析", "快速上手", combine(plan, expert_output_nvsh,
+// route_weights_nvs) -> output_sh, gathered_route_weights_sk). With row
+// weights the kernels also write each entry's weight back in token order
+// (`gathered`), so the caller needs no separate gather launch.
 #include <algorithm>
 
 #include "ep_device.cuh"
@@ -45,26 +52,44 @@ __device__ __forceinline__ uint4 pack8(const float (&acc)[8]) {
                     pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
 }
 
+// Where the weight of entry (t,k) comes from (see the file comment).
+struct Weights {
+  const float* tok;   // [N,K] per entry; NULL with rows NULL: unit weights
+  const float* rows;  // [cap] per receive row, or NULL
+  float* gathered;    // [N,K] out: rows[pos[t,k]] (0 where pos is outside
+                      // [0, cap)); written only with rows
+};
+
+// Weight of entry (t,k) whose row is p.
+__device__ __forceinline__ float entry_weight(const Weights& wt, int64_t t,
+                                              int K, int k, int32_t p,
+                                              int64_t cap) {
+  if (wt.rows) return (p >= 0 && p < cap) ? __ldg(wt.rows + p) : 0.0f;
+  return wt.tok ? __ldg(wt.tok + t * K + k) : 1.0f;
+}
+
 // KT > 0: K known at compile time; KT == 0: runtime K, in chunks of kChunk
 // terms (the chunks run in k order, so the fma order is unchanged).
 template <int KT>
 __global__ void __launch_bounds__(kCombineMaxThreads)
     k_combine(const uint16_t* __restrict__ y, const int32_t* __restrict__ pos,
-              const float* __restrict__ w, int64_t N, int Kr, int H,
-              int64_t cap, uint16_t* __restrict__ out,
-              int32_t* __restrict__ status) {
+              Weights wts, int64_t N, int Kr, int H, int64_t cap,
+              uint16_t* __restrict__ out, int32_t* __restrict__ status) {
   const int K = KT > 0 ? KT : Kr;
   const int V = H >> 3;
   for (int64_t t = blockIdx.x; t < N; t += gridDim.x) {
     const int32_t* pt = pos + t * K;
-    const float* wt = w ? w + t * K : nullptr;  // NULL: unit weights
+    if (wts.rows && wts.gathered && threadIdx.x < K) {
+      const int32_t p = __ldg(pt + threadIdx.x);
+      wts.gathered[t * K + threadIdx.x] = entry_weight(wts, t, K, threadIdx.x, p, cap);
+    }
     if constexpr (KT > 0) {
       int64_t rowoff[KT];
       float wk[KT];
 #pragma unroll
       for (int k = 0; k < KT; ++k) {
         const int32_t p = __ldg(pt + k);
-        wk[k] = w ? __ldg(wt + k) : 1.0f;
+        wk[k] = entry_weight(wts, t, K, k, p, cap);
         const bool ok = p >= 0 && p < cap;
         if (p >= cap && threadIdx.x == 0) report(status, EP_DEV_CAPACITY);
         rowoff[k] = ok ? int64_t(p) * H : int64_t(-1);
@@ -94,7 +119,7 @@ __global__ void __launch_bounds__(kCombineMaxThreads)
             wk[j] = 0.f;
             if (k0 + j < K) {
               const int32_t p = __ldg(pt + k0 + j);
-              wk[j] = w ? __ldg(wt + k0 + j) : 1.0f;
+              wk[j] = entry_weight(wts, t, K, k0 + j, p, cap);
               if (p >= 0 && p < cap) off[j] = int64_t(p) * H;
               if (p >= cap && v == threadIdx.x && threadIdx.x == 0)
                 report(status, EP_DEV_CAPACITY);
@@ -153,9 +178,8 @@ __host__ __device__ inline TmaShape tma_shape(int H, int K) {
 
 __global__ void __launch_bounds__((kTmaMaxConsumerWarps + 1) * 32, 1)
     k_combine_tma(const uint16_t* __restrict__ y, const int32_t* __restrict__ pos,
-                  const float* __restrict__ w, int64_t N, int K, int H,
-                  int64_t cap, uint16_t* __restrict__ out,
-                  int32_t* __restrict__ status) {
+                  Weights wts, int64_t N, int K, int H, int64_t cap,
+                  uint16_t* __restrict__ out, int32_t* __restrict__ status) {
   extern __shared__ __align__(128) uint8_t smem[];
   const TmaShape sh = tma_shape(H, K);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -167,15 +191,14 @@ __global__ void __launch_bounds__((kTmaMaxConsumerWarps + 1) * 32, 1)
   uint64_t* empty = full + kTmaStages;
   uint32_t* vmask = reinterpret_cast<uint32_t*>(empty + kTmaStages);
   float* wk = reinterpret_cast<float*>(vmask + kTmaStages);  // [stages][32]
-  __shared__ int s_abort;
   const int64_t units = N * sh.parts;
+  const bool forced = wait_forced(EP_WAIT_SITE_COMBINE);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTmaStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], uint32_t(cw));
     }
-    s_abort = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -189,7 +212,7 @@ __global__ void __launch_bounds__((kTmaMaxConsumerWarps + 1) * 32, 1)
     if (u < units && lane < K) {
       const int64_t t0 = u / sh.parts;
       p_n = __ldg(pos + t0 * K + lane);
-      w_n = w ? __ldg(w + t0 * K + lane) : 1.0f;
+      w_n = entry_weight(wts, t0, K, lane, p_n, cap);
     }
     for (; u < units; u += gridDim.x, ++it) {
       const int64_t t = u / sh.parts;
@@ -204,26 +227,30 @@ __global__ void __launch_bounds__((kTmaMaxConsumerWarps + 1) * 32, 1)
         if (un < units && lane < K) {
           const int64_t tn = un / sh.parts;
           p_n = __ldg(pos + tn * K + lane);
-          w_n = w ? __ldg(w + tn * K + lane) : 1.0f;
+          w_n = entry_weight(wts, tn, K, lane, p_n, cap);
         }
       }
+      if (wts.rows && wts.gathered && part == 0 && lane < K)
+        wts.gathered[t * K + lane] = wv;
       const bool valid = lane < K && p >= 0 && p < cap;
       if (lane < K && p >= cap) report(status, EP_DEV_CAPACITY);
       const unsigned m = __ballot_sync(0xffffffffu, valid);
       const int s = it % kTmaStages;
       const uint32_t ph = uint32_t(it / kTmaStages) & 1u;
       bool ok = true;
-      if (lane == 0 && it >= kTmaStages) ok = mbar_wait_bounded(&empty[s], ph ^ 1u);
+      if (lane == 0 && it >= kTmaStages) ok = mbar_wait_bounded(&empty[s], ph ^ 1u, forced);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) {
         if (lane == 0) report(status, EP_DEV_TIMEOUT);
         break;
       }
-      if (lane < 32) wk[s * 32 + lane] = wv;
-      if (lane == 0) {
-        vmask[s] = m;
-        mbar_arrive_expect_tx(&full[s], uint32_t(__popc(m)) * bytes);
-      }
+      // Every lane's weight is in shared memory before lane 0 arrives: the
+      // arrive (a release) then covers the whole warp's writes, and the
+      // consumers' wait on the phase (an acquire) sees them.
+      wk[s * 32 + lane] = wv;
+      if (lane == 0) vmask[s] = m;
+      __syncwarp();
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], uint32_t(__popc(m)) * bytes);
       __syncwarp();
       if (valid)
         bulk_g2s(in_base + size_t(s) * sh.in_bytes + size_t(lane) * sh.part_ch * 2,
@@ -251,12 +278,9 @@ __global__ void __launch_bounds__((kTmaMaxConsumerWarps + 1) * 32, 1)
       const uint32_t ph = uint32_t(it / kTmaStages) & 1u;
       uint8_t* ob = out_base + size_t(it % kTmaOutStages) * sh.out_bytes;
       bool ok = true;
-      if (lane == 0) ok = mbar_wait_bounded(&full[s], ph);
+      if (lane == 0) ok = mbar_wait_bounded(&full[s], ph, forced);
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) {
-        if (lane == 0) report(status, EP_DEV_TIMEOUT);
-        s_abort = 1;
-      }
+      if (!ok && lane == 0) report(status, EP_DEV_TIMEOUT);
       const uint32_t m = vmask[s];
       const uint8_t* st = in_base + size_t(s) * sh.in_bytes;
       for (int v = threadIdx.x; v < (len >> 3); v += nthreads) {
@@ -274,8 +298,8 @@ __global__ void __launch_bounds__((kTmaMaxConsumerWarps + 1) * 32, 1)
       fence_proxy_async_smem();
       // the other output stage must have been read by its store
       if (issuer) bulk_wait_read<0>();
-      asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
-      if (s_abort) break;
+      // every consumer warp leaves together once any of them gave up
+      if (named_barrier_or(1, nthreads, !ok)) break;
       if (issuer) {
         bulk_s2g(out + t * H + c0, ob, uint32_t(len) * 2u);
         bulk_commit();
@@ -285,7 +309,7 @@ __global__ void __launch_bounds__((kTmaMaxConsumerWarps + 1) * 32, 1)
   }
 }
 
-cudaError_t run_tma(const uint16_t* y, const int32_t* pos, const float* w,
+cudaError_t run_tma(const uint16_t* y, const int32_t* pos, const Weights& w,
                     int64_t N, int K, int H, int64_t cap, uint16_t* out,
                     int num_sms, int32_t* status, cudaStream_t stream) {
   const TmaShape sh = tma_shape(H, K);
@@ -300,7 +324,7 @@ cudaError_t run_tma(const uint16_t* y, const int32_t* pos, const float* w,
 }
 
 template <int KT>
-cudaError_t run(const uint16_t* y, const int32_t* pos, const float* w,
+cudaError_t run(const uint16_t* y, const int32_t* pos, const Weights& w,
                 int64_t N, int K, int H, int64_t cap, uint16_t* out,
                 int num_sms, int32_t* status, cudaStream_t stream) {
   const int V = H >> 3;
@@ -322,9 +346,15 @@ cudaError_t run(const uint16_t* y, const int32_t* pos, const float* w,
 
 }  // namespace
 
-cudaError_t launch_combine(const void* y_, const int32_t* pos, const float* w,
-                           int64_t N, int K, int H, int64_t cap, void* out_,
-                           int num_sms, int32_t* status, cudaStream_t stream) {
+cudaError_t set_wait_debug_combine(uint32_t sites, uint64_t budget_ns) {
+  return set_wait_debug_here(sites, budget_ns);
+}
+
+cudaError_t launch_combine(const void* y_, const int32_t* pos, const float* w_tok,
+                           const float* w_rows, float* gathered, int64_t N,
+                           int K, int H, int64_t cap, void* out_, int num_sms,
+                           int32_t* status, cudaStream_t stream) {
+  const Weights w{w_rows ? nullptr : w_tok, w_rows, w_rows ? gathered : nullptr};
   const uint16_t* y = static_cast<const uint16_t*>(y_);
   uint16_t* out = static_cast<uint16_t*>(out_);
   // The TMA pipeline needs enough (token, part) units per SM to fill its

@@ -40,10 +40,6 @@ __host__ __device__ constexpr uint32_t align128(uint32_t x) {
   return (x + 127u) & ~127u;
 }
 
-__device__ __forceinline__ void named_barrier(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 // ---------------------------------------------------------------------------
 // padding rows: zero payload, zero scales, zero weight (all warps of the grid)
 // ---------------------------------------------------------------------------
@@ -102,11 +98,13 @@ __global__ void __launch_bounds__(32)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + size_t(stages) * stage_bytes);
   const int64_t first = blockIdx.x, stride = gridDim.x;
   const int64_t n_mine = first < N ? (N - 1 - first) / stride + 1 : 0;
+  const bool forced = wait_forced(EP_WAIT_SITE_DISPATCH);
+  int64_t issued = 0;  // rows requested so far (lane 0)
 
   if (lane == 0) {
     for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
     fence_mbar_init();
-    for (int64_t i = 0; i < stages && i < n_mine; ++i) {
+    for (int64_t i = 0; i < stages && i < n_mine; ++i, ++issued) {
       mbar_arrive_expect_tx(&full[i], row_bytes);
       bulk_g2s(smem + size_t(i) * stage_bytes, hidden + (first + i * stride) * H,
                row_bytes, &full[i]);
@@ -129,7 +127,7 @@ __global__ void __launch_bounds__(32)
         p_l = -1;
       }
     }
-    if (lane == 0) ok = mbar_wait_bounded(&full[s], uint32_t(i / stages) & 1u);
+    if (lane == 0) ok = mbar_wait_bounded(&full[s], uint32_t(i / stages) & 1u, forced);
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (!ok) {
       if (lane == 0) report(status, EP_DEV_TIMEOUT);
@@ -151,15 +149,17 @@ __global__ void __launch_bounds__(32)
         mbar_arrive_expect_tx(&full[sp], row_bytes);
         bulk_g2s(smem + size_t(sp) * stage_bytes, hidden + (first + nxt * stride) * H,
                  row_bytes, &full[sp]);
+        ++issued;
       }
     }
     if (lane < K && p_l >= 0 && recv_w) recv_w[p_l] = w_l;
   }
   if (lane == 0) {
-    // Loads still in flight after a give-up, then all stores complete.
+    // Loads still in flight after a give-up (the last row requested into
+    // each stage), then all stores complete.
     if (!ok) {
-      for (int64_t i = 0; i < stages && i < n_mine; ++i) {
-        const int64_t last = n_mine - 1 - ((n_mine - 1 - i) % stages);
+      for (int64_t i = 0; i < stages && i < issued; ++i) {
+        const int64_t last = issued - 1 - ((issued - 1 - i) % stages);
         mbar_wait_bounded(&full[i], uint32_t(last / stages) & 1u);
       }
     }
@@ -197,14 +197,13 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32)
   // Bulk stores need 16-byte multiples; the scales of a row qualify when
   // H is a multiple of 512, otherwise they are stored by the lanes.
   const bool bulk_scales = (scale_bytes % 16u) == 0u;
-  __shared__ int s_abort;
+  const bool forced = wait_forced(EP_WAIT_SITE_DISPATCH);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < s_in; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], uint32_t(cw));
     }
-    s_abort = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -216,7 +215,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32)
       for (int64_t t = blockIdx.x; t < N; t += gridDim.x, ++it) {
         const int s = it % s_in;
         const uint32_t ph = uint32_t(it / s_in) & 1u;
-        if (it >= s_in && !mbar_wait_bounded(&empty[s], ph ^ 1u)) {
+        if (it >= s_in && !mbar_wait_bounded(&empty[s], ph ^ 1u, forced)) {
           report(status, EP_DEV_TIMEOUT);
           break;
         }
@@ -251,12 +250,9 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32)
         }
       }
       bool ok = true;
-      if (lane == 0) ok = mbar_wait_bounded(&full[s], ph);
+      if (lane == 0) ok = mbar_wait_bounded(&full[s], ph, forced);
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) {
-        if (lane == 0) report(status, EP_DEV_TIMEOUT);
-        s_abort = 1;
-      }
+      if (!ok && lane == 0) report(status, EP_DEV_TIMEOUT);
       const uint8_t* row = in_base + size_t(s) * in_bytes;
       for (int u = warp; u * kUnitCh < H; u += cw) {
         const int c0 = u * kUnitCh + lane * 16;  // first channel of this lane
@@ -286,8 +282,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32)
         else
           bulk_wait_read<0>();
       }
-      named_barrier(1, cw * 32);
-      if (s_abort) break;
+      // every consumer warp leaves together once any of them gave up
+      if (named_barrier_or(1, cw * 32, !ok)) break;
       // lane 0 of warp 0 issues the stores; the positions reach it through a
       // shuffle that the whole warp executes
       if (warp == 0) {
@@ -358,6 +354,10 @@ Cfg bf16_cfg(int H) {
 }
 
 }  // namespace
+
+cudaError_t set_wait_debug_dispatch(uint32_t sites, uint64_t budget_ns) {
+  return set_wait_debug_here(sites, budget_ns);
+}
 
 cudaError_t launch_dispatch(const void* hidden, const float* w,
                             const int32_t* pos, const int32_t* row_src,

@@ -30,6 +30,43 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // not been satisfied after this long reports EP_DEV_TIMEOUT and returns.
 constexpr uint64_t kWaitBudgetNs = 2000000000ull;  // 2 s
 
+// Forced give-ups (ep_debug_force_timeouts). A wait at a listed site
+// (EP_WAIT_SITE_* bits) ignores its condition, as if nothing ever set it,
+// and gives up after `budget_ns`; the kernel then takes the same give-up
+// path a real stall would. Waits for copies already in flight (the drains
+// before a CTA exits) are never forced. Each translation unit holds its own
+// copy of this word (it is static), set for the current device by that
+// unit's wait-debug setter; zero by default: nothing forced.
+struct WaitDebug {
+  uint32_t sites;
+  uint32_t reserved;
+  uint64_t budget_ns;
+};
+static __device__ WaitDebug g_wait_debug;
+
+// Read once at kernel entry by the kernels that wait at `site`.
+__device__ __forceinline__ bool wait_forced(uint32_t site) {
+  return (*reinterpret_cast<volatile const uint32_t*>(&g_wait_debug.sites) & site) != 0u;
+}
+
+__device__ __forceinline__ uint64_t forced_budget_ns() {
+  return *reinterpret_cast<volatile const uint64_t*>(&g_wait_debug.budget_ns);
+}
+
+// Spin until the forced budget runs out (the condition is never looked at).
+__device__ __forceinline__ void forced_stall() {
+  const uint64_t budget = forced_budget_ns();
+  const uint64_t t0 = globaltimer_ns();
+  while (globaltimer_ns() - t0 <= budget) {
+  }
+}
+
+// Host side: set this translation unit's copy on the current device.
+static inline cudaError_t set_wait_debug_here(uint32_t sites, uint64_t budget_ns) {
+  const WaitDebug c{sites, 0u, budget_ns};
+  return cudaMemcpyToSymbol(g_wait_debug, &c, sizeof(c));
+}
+
 // ---------------------------------------------------------------------------
 // relaxed / acquire global accesses for inter-CTA flags
 // ---------------------------------------------------------------------------
@@ -124,8 +161,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with `parity` to complete; false after the budget.
+// `forced`: a forced give-up (see WaitDebug), false after the forced budget.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar,
-                                                  uint32_t parity) {
+                                                  uint32_t parity,
+                                                  bool forced = false) {
+  if (forced) {
+    forced_stall();
+    return false;
+  }
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
@@ -180,6 +223,22 @@ __device__ __forceinline__ void grid_dependency_wait() {
 // Lets the kernel queued behind this one start launching its CTAs.
 __device__ __forceinline__ void grid_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Named barrier `id` over `nthreads` threads that also ORs `pred` over them:
+// every participant gets the same answer, so a decision taken on it (such
+// as leaving a loop that holds this barrier) is the same in every warp.
+__device__ __forceinline__ bool named_barrier_or(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(uint32_t(pred)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0u;
 }
 
 // Make generic-proxy shared-memory writes visible to the async proxy.

@@ -59,10 +59,14 @@ cudaError_t launch_dispatch(const void* hidden, const float* w,
                             int32_t* status, cudaStream_t stream,
                             bool pdl = false);
 
-// w == NULL: unit weights (dispatch backward)
-cudaError_t launch_combine(const void* y, const int32_t* pos, const float* w,
-                           int64_t N, int K, int H, int64_t cap, void* out,
-                           int num_sms, int32_t* status, cudaStream_t stream);
+// Weights: w_rows (per receive row, [cap]) when non-NULL, with each entry's
+// weight also written to `gathered` [N,K] when that is non-NULL; else w_tok
+// (per entry, [N,K]); both NULL: unit weights (dispatch backward).
+cudaError_t launch_combine(const void* y, const int32_t* pos,
+                           const float* w_tok, const float* w_rows,
+                           float* gathered, int64_t N, int K, int H,
+                           int64_t cap, void* out, int num_sms,
+                           int32_t* status, cudaStream_t stream);
 
 // ---- backward pair ---------------------------------------------------------
 
@@ -88,7 +92,7 @@ cudaError_t launch_plan_balanced(const int32_t* counts, int R, int S, int K,
 
 cudaError_t launch_prefetch(const int32_t* slot_expert, int R, int E, int B,
                             int64_t elems, void* gate, void* up, void* down,
-                            int num_sms, cudaStream_t stream);
+                            int num_sms, int32_t* status, cudaStream_t stream);
 
 cudaError_t launch_reduce_slot_grads(const int32_t* slot_expert, int R, int E,
                                      int B, int64_t elems, float* g0, float* g1,
@@ -103,6 +107,14 @@ cudaError_t launch_debug_quantize(const float* x, const float* scale,
                                   uint8_t* out, int64_t n, cudaStream_t stream);
 cudaError_t launch_debug_wait(const int32_t* flag, int64_t max_polls,
                               int32_t* status, cudaStream_t stream);
+
+// Forced give-ups of the listed wait sites (EP_WAIT_SITE_* bits) on the
+// current device, one setter per translation unit that holds wait sites.
+cudaError_t set_wait_debug_layout(uint32_t sites, uint64_t budget_ns);
+cudaError_t set_wait_debug_layout_small(uint32_t sites, uint64_t budget_ns);
+cudaError_t set_wait_debug_dispatch(uint32_t sites, uint64_t budget_ns);
+cudaError_t set_wait_debug_combine(uint32_t sites, uint64_t budget_ns);
+cudaError_t set_wait_debug_plan(uint32_t sites, uint64_t budget_ns);
 
 // SM count of the current device (cached per device).
 int device_sm_count();

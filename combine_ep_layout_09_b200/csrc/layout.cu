@@ -148,10 +148,13 @@ __global__ void __launch_bounds__(kHistThreads)
 // 2 * kLookbackWindow predecessors are covered per round of loads. Every
 // lane of the warp calls this (shuffles); `active` lanes own an expert.
 // Bounded: reports EP_DEV_TIMEOUT and returns what it has after
-// kWaitBudgetNs without progress.
+// kWaitBudgetNs without progress. `forced`: every descriptor reads as not
+// yet published, so the look-back gives up after the forced budget.
 __device__ __forceinline__ uint32_t lookback_pair(const uint32_t* desc, int E,
                                                   int e, bool active, int h,
-                                                  int tile, int32_t* status) {
+                                                  int tile, int32_t* status,
+                                                  bool forced) {
+  const uint64_t budget = forced ? forced_budget_ns() : kWaitBudgetNs;
   uint32_t excl = 0;
   int j = tile - 1;               // nearest predecessor not yet consumed
   bool done = !active || j < 0;
@@ -162,8 +165,9 @@ __device__ __forceinline__ uint32_t lookback_pair(const uint32_t* desc, int E,
     uint32_t v[kLookbackWindow];
 #pragma unroll
     for (int q = 0; q < kLookbackWindow; ++q)
-      v[q] = (!done && hi - q >= 0) ? ld_relaxed_gpu(desc + int64_t(hi - q) * E + e)
-                                    : 0u;
+      v[q] = (!done && !forced && hi - q >= 0)
+                 ? ld_relaxed_gpu(desc + int64_t(hi - q) * E + e)
+                 : 0u;
     uint32_t sum = 0;
     int used = 0;
     bool stop = false, found = false;
@@ -209,7 +213,7 @@ __device__ __forceinline__ uint32_t lookback_pair(const uint32_t* desc, int E,
         } else if (!waiting) {
           waiting = true;
           t0 = globaltimer_ns();
-        } else if (globaltimer_ns() - t0 > kWaitBudgetNs) {
+        } else if (globaltimer_ns() - t0 > budget) {
           report(status, EP_DEV_TIMEOUT);
           done = true;
         }
@@ -326,12 +330,14 @@ __device__ __forceinline__ void tile_totals_publish(int32_t* whist,
 // this one; publishes this tile's inclusive prefix. Two threads per expert.
 __device__ __forceinline__ void tile_lookback(const int32_t* tcount,
                                               int32_t* excl, int E, int tile,
-                                              uint32_t* desc, int32_t* status) {
+                                              uint32_t* desc, int32_t* status,
+                                              bool forced) {
   const int h = threadIdx.x & 1;
   for (int e0 = 0; e0 < E; e0 += kScanThreads / kLookbackPair) {
     const int e = e0 + int(threadIdx.x) / kLookbackPair;
     const bool active = e < E;
-    const uint32_t x = lookback_pair(desc, E, active ? e : 0, active, h, tile, status);
+    const uint32_t x =
+        lookback_pair(desc, E, active ? e : 0, active, h, tile, status, forced);
     if (active && h == 0) {
       if (tile > 0)
         st_relaxed_gpu(desc + int64_t(tile) * E + e,
@@ -347,12 +353,14 @@ __device__ __forceinline__ void tile_lookback(const int32_t* tcount,
 // entries of e in the tiles before this one, tot[e] = in all tiles. P
 // threads share an expert, each summing tiles j = p, p+P, ... with
 // kReduceBatch loads in flight; the P partial sums meet in `scratch`
-// ([2][P][E] ints).
+// ([2][P][E] ints). `forced`: every descriptor stays pending, so the wait
+// gives up after the forced budget.
 constexpr int kReduceBatch = 16;
 __device__ __forceinline__ void tile_reduce(const uint32_t* desc, int E, int tile,
                                             int num_tiles, int32_t* excl,
                                             int32_t* tot, int32_t* scratch,
-                                            int32_t* status) {
+                                            int32_t* status, bool forced) {
+  const uint64_t budget = forced ? forced_budget_ns() : kWaitBudgetNs;
   const int P = max(1, min(32, kScanThreads / E));
   for (int idx = threadIdx.x; idx < E * P; idx += kScanThreads) {
     const int e = idx % E, p = idx / E;
@@ -366,7 +374,7 @@ __device__ __forceinline__ void tile_reduce(const uint32_t* desc, int E, int til
         v[q] = kFlagAggregate;
         if (j < num_tiles) {
           v[q] = ld_relaxed_gpu(desc + int64_t(j) * E + e);
-          if ((v[q] & ~kValueMask) == 0u) pending |= 1u << q;
+          if ((v[q] & ~kValueMask) == 0u || forced) pending |= 1u << q;
         }
       }
       if (pending) {  // some tile has not published yet: poll those
@@ -376,9 +384,9 @@ __device__ __forceinline__ void tile_reduce(const uint32_t* desc, int E, int til
           for (int q = 0; q < kReduceBatch; ++q)
             if ((pending >> q) & 1u) {
               v[q] = ld_relaxed_gpu(desc + int64_t(j0 + q * P) * E + e);
-              if ((v[q] & ~kValueMask) != 0u) pending &= ~(1u << q);
+              if ((v[q] & ~kValueMask) != 0u && !forced) pending &= ~(1u << q);
             }
-          if (pending && globaltimer_ns() - t0 > kWaitBudgetNs) {
+          if (pending && globaltimer_ns() - t0 > budget) {
             report(status, EP_DEV_TIMEOUT);
             break;
           }
@@ -510,6 +518,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   __shared__ int s_tile;
   __shared__ int32_t s_warp[kScanThreads / 32];
   const int tid = threadIdx.x, warp = tid >> 5;
+  const bool forced = wait_forced(EP_WAIT_SITE_LOOKBACK);
 
   // Tiles are claimed in order of arrival, so every predecessor of a tile
   // belongs to a CTA that is already running: the look-back progresses.
@@ -523,7 +532,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   rank_in_warps(topk, M, E, wbase, my, kr);
   __syncthreads();
   tile_totals_publish(sm.whist, sm.tcnt, sm.part, E, tile, desc);
-  tile_lookback(sm.tcnt, sm.base, E, tile, desc, status);
+  tile_lookback(sm.tcnt, sm.base, E, tile, desc, status, forced);
   tile_prefix(sm.tcnt, sm.tpre, E, s_warp);
   for (int e = tid; e < E; e += kScanThreads) sm.base[e] += __ldg(offsets + e);
   __syncthreads();
@@ -547,6 +556,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   __shared__ int32_t s_warp2[2 * kScanThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int tile = blockIdx.x;
+  const bool forced = wait_forced(EP_WAIT_SITE_TILE_REDUCE);
 
   for (int j = tid; j < kScanWarps * E; j += kScanThreads) sm.whist[j] = 0;
   __syncthreads();
@@ -558,7 +568,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   __syncthreads();
   // counts published as aggregates only; every tile then reads all of them
   tile_totals_publish(sm.whist, sm.tcnt, sm.part, E, tile, desc, false);
-  tile_reduce(desc, E, tile, num_tiles, sm.base, sm.tot, sm.sorted, status);
+  tile_reduce(desc, E, tile, num_tiles, sm.base, sm.tot, sm.sorted, status, forced);
   // each tile scans the padded totals into expert offsets and its own counts
   // into its counting-sort prefix, in one pass
   for (int e = tid; e < E; e += kScanThreads) {
@@ -627,6 +637,10 @@ int fused_capacity(int E) {
 }
 
 }  // namespace
+
+cudaError_t set_wait_debug_layout(uint32_t sites, uint64_t budget_ns) {
+  return set_wait_debug_here(sites, budget_ns);
+}
 
 size_t layout_workspace_bytes(int64_t entries, int E) {
   const int64_t tiles = (entries + kScanTile - 1) / kScanTile;

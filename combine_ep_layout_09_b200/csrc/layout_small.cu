@@ -92,9 +92,9 @@ __host__ __device__ inline SmallPlan small_plan(int64_t N, int K, int E, int H,
 
 // Bounded wait of lane 0 on `bar`, the verdict shared by the warp.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
-                                          int32_t* status) {
+                                          int32_t* status, bool forced) {
   bool ok = true;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait_bounded(bar, parity);
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait_bounded(bar, parity, forced);
   ok = __shfl_sync(0xffffffffu, ok, 0);
   if (!ok && (threadIdx.x & 31) == 0) report(status, EP_DEV_TIMEOUT);
   return ok;
@@ -310,6 +310,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
   __shared__ int s_next;  // next FP8 (token, unit) pair to quantise
   __shared__ int32_t s_warp[kSmallWarps];
   const int units = (H + kQuantUnit - 1) / kQuantUnit;
+  const bool forced = wait_forced(EP_WAIT_SITE_SMALL);
 
   int issued = 0;  // rows requested (thread 0 requests them all)
   auto load_row = [&](int j) {
@@ -399,8 +400,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
         if (idx >= n_mine * units || s_abort) break;
         const int j = idx / units, u = idx - j * units;
         const int s = j % nb, m = j / nb;
-        bool ok = warp_wait(&full[s], uint32_t(m) & 1u, status);
-        if (ok && m >= 1) ok = warp_wait(&ofree[s], uint32_t(m - 1) & 1u, status);
+        bool ok = warp_wait(&full[s], uint32_t(m) & 1u, status, forced);
+        if (ok && m >= 1) ok = warp_wait(&ofree[s], uint32_t(m - 1) & 1u, status, forced);
         if (!ok) {
           s_abort = 1;
           break;
@@ -421,7 +422,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
       const int lag = nb >= 2 ? 1 : 0;  // tokens whose stores may still read
       for (int j = 0; j < n_mine; ++j) {
         const int s = j % nb, m = j / nb;
-        if (!warp_wait(&qdone[s], uint32_t(m) & 1u, status)) {
+        if (!warp_wait(&qdone[s], uint32_t(m) & 1u, status, forced)) {
           s_abort = 1;
           break;
         }
@@ -461,11 +462,16 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
     }
   } else if constexpr (kMode == Copy::kBf16) {
     const bool issuer = lane < K;  // lane k of a warp stores row k
+    bool gave_up = false;
     for (int b0 = 0; b0 < n_mine; b0 += nb) {
       const int n = min(nb, n_mine - b0);
       for (int jj = warp; jj < n; jj += kSmallWarps) {
         const int j = b0 + jj;
-        if (!warp_wait(&full[jj], uint32_t(j / nb) & 1u, status)) continue;
+        if (!warp_wait(&full[jj], uint32_t(j / nb) & 1u, status, forced)) {
+          s_abort = 1;  // its load may still be in flight: drained at the end
+          gave_up = true;
+          continue;
+        }
         if (issuer) {
           const int p = spos[j * K + lane];
           if (p >= 0)
@@ -475,9 +481,11 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
       }
       if (issuer) bulk_commit();
       if (b0 + n < n_mine) {
-        // the next batch reuses the stages once these stores have read them
+        // the next batch reuses the stages once these stores have read them;
+        // after a give-up in any warp, no further batch is loaded (the
+        // decision is the barrier's, hence the same in every warp)
         if (issuer) bulk_wait_read<0>();
-        __syncthreads();
+        if (__syncthreads_or(gave_up)) break;
         if (tid == 0)
           for (int j = b0 + n; j < b0 + n + nb && j < n_mine; ++j) load_row(j);
       }
@@ -542,6 +550,10 @@ cudaError_t run_small(const int32_t* topk, int64_t N, int K, int E, int pad,
 }
 
 }  // namespace
+
+cudaError_t set_wait_debug_layout_small(uint32_t sites, uint64_t budget_ns) {
+  return set_wait_debug_here(sites, budget_ns);
+}
 
 bool small_layout_fits(int64_t N, int K, int E, int H, int copy, int num_sms) {
   if (N * K > kSmallMaxEntries) return false;

@@ -188,7 +188,8 @@ constexpr int kMaxSlotList = 1024;
 __global__ void __launch_bounds__(32)
     k_prefetch_tma(const int32_t* __restrict__ slot_expert, int RB, int E,
                    int64_t row_bytes, uint8_t* __restrict__ gate,
-                   uint8_t* __restrict__ up, uint8_t* __restrict__ down) {
+                   uint8_t* __restrict__ up, uint8_t* __restrict__ down,
+                   int32_t* __restrict__ status) {
   extern __shared__ __align__(128) uint8_t smb[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smb + kTmaCopyStages * kTmaChunk);
   int32_t* list = reinterpret_cast<int32_t*>(full + kTmaCopyStages);  // (slot, e)
@@ -228,9 +229,11 @@ __global__ void __launch_bounds__(32)
     *src = W + int64_t(list[2 * j + 1]) * row_bytes + off;
     *dst = W + (int64_t(E) + list[2 * j]) * row_bytes + off;
   };
+  const bool forced = wait_forced(EP_WAIT_SITE_PREFETCH);
+  int64_t issued = 0;  // units whose load has been requested, in order
   for (int s = 0; s < kTmaCopyStages; ++s) mbar_init(&full[s], 1);
   fence_mbar_init();
-  for (int64_t i = 0; i < kTmaCopyStages && i < n_mine; ++i) {
+  for (int64_t i = 0; i < kTmaCopyStages && i < n_mine; ++i, ++issued) {
     const uint8_t* src;
     uint8_t* dst;
     uint32_t bytes;
@@ -244,7 +247,10 @@ __global__ void __launch_bounds__(32)
     uint8_t* dst;
     uint32_t bytes;
     unit(i, &src, &dst, &bytes);
-    if (!mbar_wait_bounded(&full[s], uint32_t(i / kTmaCopyStages) & 1u)) break;
+    if (!mbar_wait_bounded(&full[s], uint32_t(i / kTmaCopyStages) & 1u, forced)) {
+      report(status, EP_DEV_TIMEOUT);
+      break;
+    }
     bulk_s2g(dst, smb + size_t(s) * kTmaChunk, bytes);
     bulk_commit();
     const int64_t nxt = i - 1 + kTmaCopyStages;
@@ -254,11 +260,13 @@ __global__ void __launch_bounds__(32)
       unit(nxt, &src, &dst, &bytes);
       mbar_arrive_expect_tx(&full[sp], bytes);
       bulk_g2s(smb + size_t(sp) * kTmaChunk, src, bytes, &full[sp]);
+      ++issued;
     }
   }
-  // drain: loads in flight after a give-up, then every store
-  for (int64_t i = 0; i < kTmaCopyStages && i < n_mine; ++i) {
-    const int64_t last = n_mine - 1 - ((n_mine - 1 - i) % kTmaCopyStages);
+  // drain: the last load requested into each stage (still in flight after a
+  // give-up), then every store
+  for (int64_t i = 0; i < kTmaCopyStages && i < issued; ++i) {
+    const int64_t last = issued - 1 - ((issued - 1 - i) % kTmaCopyStages);
     mbar_wait_bounded(&full[i], uint32_t(last / kTmaCopyStages) & 1u);
   }
   bulk_wait_all<0>();
@@ -399,9 +407,13 @@ cudaError_t launch_plan_balanced(const int32_t* counts, int R, int S, int K,
   return cudaGetLastError();
 }
 
+cudaError_t set_wait_debug_plan(uint32_t sites, uint64_t budget_ns) {
+  return set_wait_debug_here(sites, budget_ns);
+}
+
 cudaError_t launch_prefetch(const int32_t* slot_expert, int R, int E, int B,
                             int64_t elems, void* gate, void* up, void* down,
-                            int num_sms, cudaStream_t stream) {
+                            int num_sms, int32_t* status, cudaStream_t stream) {
   const int64_t RB = int64_t(R) * B;
   if (RB == 0 || elems == 0) return cudaSuccess;
   if (RB <= kMaxSlotList) {
@@ -417,7 +429,7 @@ cudaError_t launch_prefetch(const int32_t* slot_expert, int R, int E, int B,
     const int grid = num_sms * std::max(1, per_sm);
     k_prefetch_tma<<<grid, 32, smem, stream>>>(
         slot_expert, int(RB), E, elems * 2, static_cast<uint8_t*>(gate),
-        static_cast<uint8_t*>(up), static_cast<uint8_t*>(down));
+        static_cast<uint8_t*>(up), static_cast<uint8_t*>(down), status);
     return cudaGetLastError();
   }
   const int64_t vecs = elems * 2 / 16;

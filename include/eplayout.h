@@ -129,10 +129,15 @@ EP_API int ep_layout(const int32_t* topk_experts, int R, int S, int K, int E,
  * on a GPU until the process exits. Nothing is allocated by the call.
  *   - Limit: problems with ep_layout_workspace_bytes(R*S, K, E) larger than
  *     EP_LAYOUT_STATIC_SCRATCH_BYTES are refused with EP_ERR_WORKSPACE
- *     before any CUDA call (E=256 fits up to about 16 M entries N*K).
+ *     before any CUDA call. That size is 256 + align256(4E) +
+ *     ceil(N*K/4096) * 4E bytes: E=256 fits up to N*K = 4,186,112 entries
+ *     (1022 tiles of 4096), E=64 up to 16,366,592.
  *   - The first call on each GPU looks up the array's device address
- *     (cudaGetSymbolAddress, with that GPU current) and caches it; make that
- *     first call before any stream capture.
+ *     (cudaGetSymbolAddress, with that GPU current) and caches it together
+ *     with the unique id of the context it was found in; a call in another
+ *     context (after cudaDeviceReset, for instance) looks it up again. Make
+ *     the first call on a GPU, and the first after its context changed,
+ *     before any stream capture.
  *   - All calls on a GPU share the array and it keeps the last call's
  *     contents. Each call clears what must start at zero, but two calls that
  *     overlap on the GPU (different streams, unordered host threads) race
@@ -237,6 +242,33 @@ EP_API int ep_combine(const void* expert_out, const int32_t* pos,
                const float* route_weights, int64_t num_tokens, int K, int H,
                int64_t cap, void* out, int num_sms, int32_t* status,
                void* stream);
+
+/*
+ * ep_combine_recv_weights -- ep_combine with the weights taken on the
+ * receive side, as in the pages' combine(plan, expert_output_nvsh,
+ * route_weights_nvs) -> output_sh, gathered_route_weights_sk
+ * ("MoonEP核心功能深度剖析", "快速上手"): the weight of entry (t,k) is
+ * recv_weights[pos[t,k]], the per-row weight ep_dispatch wrote, and the
+ * call also hands those weights back in token order. One launch: the
+ * gather rides on the combine's own reads of pos.
+ *
+ * in   expert_out        bf16 [cap, H]
+ *      pos               int32 [N, K] (entries outside [0, cap) skipped)
+ *      recv_weights      fp32 [cap]
+ * out  out               bf16 [N, H], as ep_combine with
+ *                        w[t,k] = recv_weights[pos[t,k]] (bit-identical to
+ *                        ep_combine with the token-side weights dispatch
+ *                        copied, since those are the same values)
+ *      gathered_route_weights  fp32 [N, K] or NULL: recv_weights[pos[t,k]],
+ *                        0 where pos[t,k] is outside [0, cap)
+ *      num_sms, status   as for ep_combine
+ */
+EP_API int ep_combine_recv_weights(const void* expert_out, const int32_t* pos,
+                                   const float* recv_weights,
+                                   int64_t num_tokens, int K, int H,
+                                   int64_t cap, void* out,
+                                   float* gathered_route_weights, int num_sms,
+                                   int32_t* status, void* stream);
 
 /*
  * ep_dispatch_backward -- gradient of the bf16 dispatch with respect to the
@@ -347,10 +379,12 @@ EP_API int ep_plan_balanced(const int32_t* tokens_per_expert, int R, int S, int 
  *                        E + d*B + b <- row slot_expert[d,b] when that is
  *                        >= 0; every other row is left as it is
  *      num_sms           SMs to use, 0 = all
+ *      status            EP_DEV_TIMEOUT may be OR-ed in
  */
 EP_API int ep_prefetch_weights(const int32_t* slot_expert, int R, int E, int B,
                         int64_t elems_per_expert, void* gate, void* up,
-                        void* down, int num_sms, void* stream);
+                        void* down, int num_sms, int32_t* status,
+                        void* stream);
 
 /*
  * ep_reduce_slot_grads -- fold the gradients of the prefetched expert copies
@@ -393,6 +427,33 @@ EP_API int ep_debug_quantize(const float* x, const float* group_scale,
  * exercised with a flag that nothing sets. */
 EP_API int ep_debug_bounded_wait(const int32_t* flag, int64_t max_polls,
                           int32_t* status, void* stream);
+
+/* Wait sites of the shipped kernels, for ep_debug_force_timeouts. */
+#define EP_WAIT_SITE_LOOKBACK 1u    /* layout, two-kernel path: look-back over
+                                       the earlier tiles' published counts */
+#define EP_WAIT_SITE_TILE_REDUCE 2u /* layout, cooperative path: wait until
+                                       every tile has published its counts */
+#define EP_WAIT_SITE_DISPATCH 4u    /* dispatch kernels: token row landed in
+                                       shared memory / stage free again */
+#define EP_WAIT_SITE_COMBINE 8u     /* large-batch combine: gathered part-rows
+                                       landed / stage free again */
+#define EP_WAIT_SITE_SMALL 16u      /* one-launch layout + dispatch: row
+                                       landed / quantised / output read */
+#define EP_WAIT_SITE_PREFETCH 32u   /* weight prefetch: chunk landed */
+#define EP_WAIT_SITE_ALL 63u
+
+/* Make every wait at the listed sites give up, on the current device, for
+ * the launches that follow: such a wait ignores its condition, as if nothing
+ * ever set it, spins for budget_ns (0 < budget_ns <= 2e9) and then takes the
+ * kernel's give-up path (EP_DEV_TIMEOUT OR-ed into *status, the kernel
+ * returns; outputs are then undefined but every access stays in bounds).
+ * Waits for copies already in flight, which a CTA drains before it exits,
+ * are never forced. sites = 0 restores normal operation (budget_ns is then
+ * ignored). The setting is
+ * written with synchronous copies to the device, so call it outside stream
+ * capture and with no launch of this library in flight. For tests of the
+ * give-up paths: a stall is made without any GPU fault or hang. */
+EP_API int ep_debug_force_timeouts(uint32_t sites, int64_t budget_ns);
 
 #ifdef __cplusplus
 }

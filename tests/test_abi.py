@@ -41,7 +41,7 @@ def test_library_is_the_in_tree_build():
 
 
 def test_pure_host_entry_points():
-    assert ep.ep_abi_version() == 3
+    assert ep.ep_abi_version() == 4
     assert ep.ep_capacity_bound(32768, 8, 256, 128) == 32768 * 8 + 256 * 127
     assert ep.ep_capacity_bound(10, 2, 4, 1) == 20
     assert ep.ep_capacity_bound(-1, 2, 4, 1) < 0
@@ -141,16 +141,29 @@ def test_plan_prefetch_reject_on_host():
     P, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
     lib.ep_plan_balanced.argtypes = [P, i32, i32, i32, i32, i32, P, P, P, P,
                                      P, P, P]
-    lib.ep_prefetch_weights.argtypes = [P, i32, i32, i32, i64, P, P, P, i32, P]
+    lib.ep_prefetch_weights.argtypes = [P, i32, i32, i32, i64, P, P, P, i32, P,
+                                        P]
     ok = ctypes.c_void_p(1 << 20)
     assert lib.ep_plan_balanced(ok, 0, 4, 2, 8, 1, ok, ok, ok, ok, ok, None,
                                 None) == ep.EP_ERR_INVALID_ARG
     assert lib.ep_plan_balanced(ok, 2, 4, 2, 8, 1, ok, ok, ok, ok, None, None,
                                 None) == ep.EP_ERR_ALIGNMENT
-    assert lib.ep_prefetch_weights(ok, 2, 8, 1, 7, ok, ok, ok, 0,
+    assert lib.ep_prefetch_weights(ok, 2, 8, 1, 7, ok, ok, ok, 0, None,
                                    None) == ep.EP_ERR_INVALID_ARG
-    assert lib.ep_prefetch_weights(ok, 2, 8, 0, 8, ok, ok, ok, 0,
+    assert lib.ep_prefetch_weights(ok, 2, 8, 0, 8, ok, ok, ok, 0, None,
                                    None) == ep.EP_OK
+    assert lib.ep_prefetch_weights(ok, 2, 8, 1, 8, ok, ok, ok, 0,
+                                   ctypes.c_void_p(2), None) == ep.EP_ERR_ALIGNMENT
+
+
+def test_force_timeouts_rejects_on_host():
+    lib = _raw()
+    lib.ep_debug_force_timeouts.argtypes = [ctypes.c_uint32, ctypes.c_int64]
+    assert lib.ep_debug_force_timeouts(64, 1000) == ep.EP_ERR_INVALID_ARG
+    assert lib.ep_debug_force_timeouts(ep.EP_WAIT_SITE_DISPATCH, 0) == \
+        ep.EP_ERR_INVALID_ARG
+    assert lib.ep_debug_force_timeouts(ep.EP_WAIT_SITE_DISPATCH,
+                                       3_000_000_000) == ep.EP_ERR_INVALID_ARG
 
 
 def test_binding_rejects_host_tensors():
@@ -164,3 +177,19 @@ def test_binding_rejects_host_tensors():
     with pytest.raises(ValueError):
         ep.ep_layout_dispatch(t, h, wt, 1, 4, 2, 2, 8, 1, False, t, t, t, t,
                               h, workspace=torch.zeros(64, dtype=torch.uint8))
+
+
+def test_static_layout_refuses_beyond_its_array_on_host():
+    # refused before any CUDA call, so this runs without a GPU: with E=256
+    # the 1 MiB array holds 1022 tiles of 4096 entries, and one entry more
+    # needs a 1023rd
+    lib = _raw()
+    P, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    lib.ep_layout_static.argtypes = [P, i32, i32, i32, i32, i32, P, P, P, P,
+                                     i64, P, P]
+    E, limit = 256, 1022 * 4096
+    assert ep.ep_layout_workspace_bytes(limit, 1, E) <= 1 << 20
+    assert ep.ep_layout_workspace_bytes(limit + 1, 1, E) > 1 << 20
+    ok = ctypes.c_void_p(1 << 20)
+    assert lib.ep_layout_static(ok, 1, limit + 1, 1, E, 1, ok, ok, ok, ok,
+                                limit + 1, None, None) == ep.EP_ERR_WORKSPACE

@@ -5,10 +5,10 @@ import numpy as np
 import pytest
 import torch
 
+import combine_ep_layout_09_b200 as ep
 import oracle
 import workloads
-from gpu_util import (DEV, gpu_combine, gpu_layout, rows_to_host, to_bf16_dev,
-                      to_dev, u16)
+from gpu_util import gpu_combine, to_bf16_dev, to_dev, u16
 
 pytestmark = pytest.mark.gpu
 
@@ -80,26 +80,6 @@ def test_k_order_and_fma_cases():
     assert as_f32(got)[0, 0] == 2.0 ** -30
 
 
-@pytest.mark.parametrize("name", ["prefill", "decode"])
-def test_full_size_sampled(name):
-    wl = workloads.WORKLOADS[name]
-    topk, w = workloads.routing(wl)
-    g = gpu_layout(topk, wl.R, wl.S, wl.E, 1)
-    cap = g["dev"]["cap"]
-    y = workloads.expert_outputs(cap, wl.H, wl.seed, device="cuda:0")
-    out, st = gpu_combine(y, g["dev"]["pos"], to_dev(w), wl.N, wl.K)
-    assert st == 0
-    o_lay = oracle.layout(topk, wl.E, 1, cap)
-    rng = np.random.default_rng(1)
-    toks = np.sort(rng.choice(wl.N, min(wl.N, 512), replace=False))
-    toks[0], toks[-1] = 0, wl.N - 1
-    rows = o_lay["pos"][toks].ravel()
-    ysel = rows_to_host(y, rows)
-    pos_small = np.arange(len(rows), dtype=np.int32).reshape(len(toks), wl.K)
-    ref = oracle.combine(ysel, pos_small, w[toks])
-    np.testing.assert_array_equal(rows_to_host(out, toks), ref)
-
-
 @pytest.mark.parametrize("N,K,H,rows", [
     (2500, 8, 7176, 4000),    # two parts per row, the last one shorter
     (5000, 3, 520, 6000),     # one part per row
@@ -127,3 +107,33 @@ def test_widest_row_and_k32():
     pos = rng.integers(0, 600, size=(2600, 32)).astype(np.int32)
     w = rng.random((2600, 32)).astype(np.float32) / 32
     check(y, pos, w)
+
+
+@pytest.mark.parametrize("N,K,H,rows", [
+    (300, 8, 7168, 3000),     # register-gather kernel, K = 8
+    (200, 5, 520, 1500),      # runtime-K kernel
+    (2500, 8, 1024, 9000),    # bulk-copy pipeline
+    (2400, 8, 7176, 4000),    # bulk-copy pipeline, two parts per row
+])
+def test_receive_side_weights(N, K, H, rows):
+    # weight of (t,k) = recv_weights[pos[t,k]], handed back in token order
+    rng = np.random.default_rng(N * K + H)
+    y = u16(workloads.bf16_normal((rows, H), N + 7))
+    pos = rng.integers(0, rows, size=(N, K)).astype(np.int32)
+    pos[rng.random(pos.shape) < 0.05] = -1
+    rw = rng.standard_normal(rows).astype(np.float32)
+    gw_ref = oracle.gather_row_values(rw, pos)
+    out = torch.full((N, H), 0x7FBF, dtype=torch.int16,
+                     device="cuda:0").view(torch.bfloat16)
+    gathered = torch.full((N, K), -7.0, dtype=torch.float32, device="cuda:0")
+    st = torch.zeros(4, dtype=torch.int32, device="cuda:0")
+    ep.ep_combine_recv_weights(to_bf16_dev(y), to_dev(pos), to_dev(rw), N, K,
+                               H, out, gathered, status=st)
+    assert int(st[0].item()) == 0
+    np.testing.assert_array_equal(gathered.cpu().numpy(), gw_ref)
+    np.testing.assert_array_equal(u16(out), oracle.combine(y, pos, gw_ref))
+    # without the gathered output: the same result
+    out2 = torch.empty_like(out)
+    ep.ep_combine_recv_weights(to_bf16_dev(y), to_dev(pos), to_dev(rw), N, K,
+                               H, out2, None)
+    assert torch.equal(out2.view(torch.int16), out.view(torch.int16))

@@ -4,9 +4,12 @@ runtime that forbids allocation on its serving path, code running during a
 global-mode graph capture). Its scratch is a fixed array inside the library.
 
 Checked through the C ABI against ep_layout with a caller-provided workspace
-on two calls in a row with different inputs, so anything the first call left
-in the shared array would show up in the second. Results must be bit-exact,
-as for every layout test. This file is collected last on purpose.
+on two calls in a row with different inputs and sizes, both large enough to
+use the array (the cooperative kernel and the histogram + look-back pair), so
+anything the first call left in the shared array would show up in the
+second; and at the array's size limit, where the largest accepted problem
+runs and one entry more is refused. Results must be bit-exact, as for every
+layout test. This file is collected last on purpose.
 """
 import ctypes
 
@@ -61,14 +64,23 @@ def _run_workspace(topk, R, S, K, E, pad, cap):
 
 
 @pytest.mark.parametrize("first,second", [
-    # (R, S, K, E, pad): a large call followed by a smaller one, and back
-    ((8, 4096, 8, 256, 1), (4, 300, 6, 64, 16)),
-    ((4, 300, 6, 64, 16), (8, 2048, 8, 256, 128)),
+    # (R, S, K, E, pad). Every call here has more than 32768 entries, so it
+    # uses the array (smaller batches take a kernel that needs no scratch).
+    # Cooperative layout (64 tiles, E=256), then another with E=64 and
+    # padding: the second reads descriptors the first left behind.
+    ((8, 4096, 8, 256, 1), (8, 2048, 8, 64, 128)),
+    # Cooperative, then 700 tiles at E=256 (more than can be resident):
+    # the histogram + look-back path runs on the array after a fused call.
+    ((8, 4096, 8, 256, 1), (8, 44800, 8, 256, 1)),
+    # The other way round, with a different E.
+    ((8, 44800, 8, 256, 4), (4, 3000, 8, 32, 1)),
 ])
 def test_static_scratch_matches_workspace_entry_point(first, second):
     f = _static_fn()
     rng = np.random.default_rng(sum(first) + sum(second))
     for (R, S, K, E, pad) in (first, second):
+        assert R * S * K > 32768
+        assert ep.ep_layout_workspace_bytes(R * S, K, E) <= SCRATCH_BYTES
         topk = torch.from_numpy(
             rng.integers(0, E, size=(R * S, K)).astype(np.int32)).to(DEV)
         cap = ep.ep_capacity_bound(R * S, K, E, pad)
@@ -78,6 +90,30 @@ def test_static_scratch_matches_workspace_entry_point(first, second):
         for k in ("counts", "offsets", "pos", "row_src", "status"):
             assert torch.equal(a[k], b[k]), k
         assert int(a["status"][0].item()) == 0
+
+
+def test_static_scratch_at_its_size_limit():
+    # E=256: 256 + 1024 + tiles * 1024 bytes, so 1022 tiles of 4096 entries
+    # (N*K = 4,186,112) is the largest problem the 1 MiB array holds
+    f = _static_fn()
+    R, S, K, E, pad = 8, 65408, 8, 256, 1
+    assert R * S * K == 1022 * 4096
+    assert ep.ep_layout_workspace_bytes(R * S, K, E) <= SCRATCH_BYTES
+    assert ep.ep_layout_workspace_bytes(R * S * K + 1, 1, E) > SCRATCH_BYTES
+    rng = np.random.default_rng(12)
+    topk = torch.from_numpy(
+        rng.integers(0, E, size=(R * S, K)).astype(np.int32)).to(DEV)
+    cap = ep.ep_capacity_bound(R * S, K, E, pad)
+    a = _run_static(f, topk, R, S, K, E, pad, cap)
+    b = _run_workspace(topk, R, S, K, E, pad, cap)
+    torch.cuda.synchronize()
+    for k in ("counts", "offsets", "pos", "row_src", "status"):
+        assert torch.equal(a[k], b[k]), k
+    # one entry more needs a 1023rd tile: refused before any CUDA call
+    p = topk.data_ptr()
+    rc = f(p, 1, R * S * K + 1, 1, E, 1, p, p, p, p, R * S * K + 1, p,
+           torch.cuda.current_stream().cuda_stream)
+    assert rc == ep.EP_ERR_WORKSPACE
 
 
 def test_static_scratch_refuses_problems_beyond_its_size():
