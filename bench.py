@@ -18,6 +18,7 @@ logical ranks on one GPU, so the scaling is weak.
 from __future__ import annotations
 
 import argparse
+import contextlib
 import hashlib
 import json
 import os
@@ -133,7 +134,7 @@ def total_value_gbs(bytes_per_step: int, steps: int, world: int,
 
 
 class ClockSampler:
-    """Samples SM clock and throttle reasons with NVML every 10 ms."""
+    """Samples SM clock and throttle reasons with NVML every millisecond."""
 
     REASONS = {
         0x1: "gpu_idle", 0x2: "applications_clocks_setting",
@@ -174,7 +175,7 @@ class ClockSampler:
                     nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
             except Exception:
                 pass
-            time.sleep(0.01)
+            time.sleep(0.001)
 
     def __enter__(self):
         if self.nv is not None:
@@ -228,6 +229,23 @@ def layout_dispatch_kernels(wl, sms=148):
         return 1
     tiles = -(-entries // 4096)
     return (1 if tiles <= sms else 2) + 1
+
+
+def combine_kernel(wl, sms=148):
+    """Kernel one ep_combine launch runs, by the library's size rule: the
+    bulk-copy pipeline k_combine_tma when the row splits into parts whose K
+    part-rows fill a stage of at most 64 KB, its shared memory stays within
+    200 KB, and there are at least 16 (token, part) units per SM; else the
+    register gather k_combine<K>."""
+    al = lambda x: (x + 127) & ~127  # noqa: E731
+    max_ch = max(8, (65536 // (wl.K * 2)) & ~7)
+    parts = -(-wl.H // max_ch)
+    part_ch = (-(-wl.H // parts) + 7) & ~7
+    smem = (3 * al(wl.K * part_ch * 2) + 2 * al(part_ch * 2) +
+            3 * (16 + 4 + 4 * 32) + 64)
+    if smem <= 200 * 1024 and wl.N * parts >= 16 * sms:
+        return "k_combine_tma"
+    return f"k_combine<{wl.K}>"
 
 
 class Path:
@@ -380,6 +398,276 @@ class Path:
                 self.reduce_slot_grads(io)
 
 
+@contextlib.contextmanager
+def nvtx(name: str):
+    """NVTX range around a phase of the benchmark (seen by nsys / ncu)."""
+    torch.cuda.nvtx.range_push(name)
+    try:
+        yield
+    finally:
+        torch.cuda.nvtx.range_pop()
+
+
+def capture(fn, n):
+    """One CUDA graph of n calls of fn (the library allocates nothing and
+    never synchronises, so its calls capture as they are)."""
+    cs = torch.cuda.Stream()
+    cs.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cs):
+        for i in range(n):
+            fn(i)
+    torch.cuda.synchronize()
+    return g
+
+
+def replay_ms(g):
+    a_, b_ = (torch.cuda.Event(enable_timing=True),
+              torch.cuda.Event(enable_timing=True))
+    a_.record()
+    g.replay()
+    b_.record()
+    torch.cuda.synchronize()
+    return a_.elapsed_time(b_)
+
+
+def step_bytes(path, backward):
+    """Algorithmic bytes of one step of `path` and of each of its calls
+    (after a warm-up step: padding makes the used rows data-dependent)."""
+    wl = path.wl
+    used = int(path.offsets[-1].item())
+    n_slots = int((path.plan["slot"] >= 0).sum().item()) if wl.B else 0
+    b = {"layout": bytes_layout(wl.N, wl.K, wl.E, used),
+         "dispatch": bytes_dispatch(wl.N, wl.K, wl.H, wl.fp8, used),
+         "combine": bytes_combine(wl.N, wl.K, wl.H),
+         "plan_prefetch": bytes_prefetch(n_slots, wl.H, wl.I) if wl.B else 0,
+         "combine_backward": (bytes_combine_backward(wl.N, wl.K, wl.H, used)
+                              if backward else 0),
+         "dispatch_backward": (bytes_dispatch_backward(wl.N, wl.K, wl.H)
+                               if backward else 0),
+         "reduce_slot_grads": (bytes_reduce_slot_grads(
+             path.plan["slot"].cpu().numpy(), wl.H, wl.I)
+             if backward and wl.B else 0),
+         "used_rows": used}
+    b["layout_dispatch"] = b["layout"] + b["dispatch"]
+    b["step"] = (b["layout_dispatch"] + b["combine"] + b["plan_prefetch"] +
+                 b["combine_backward"] + b["dispatch_backward"] +
+                 b["reduce_slot_grads"])
+    return b
+
+
+def percentiles(us):
+    return {"p10": round(float(np.percentile(us, 10)), 2),
+            "p50": round(float(np.percentile(us, 50)), 2),
+            "p90": round(float(np.percentile(us, 90)), 2),
+            "calls": len(us)}
+
+
+def measure(paths, K, warmup, backward, device_index, flush, barrier=None,
+            rank_max=None, kernels=True):
+    """Time one workload on the input sets `paths` (one Path each).
+
+    The K timed steps are captured once into a CUDA graph and replayed once,
+    so no host launch gap sits between kernels; step i runs on input set
+    i % len(paths), so that with several sets a set's data has left the
+    126 MB L2 before it is used again. Each call's own average comes the
+    same way from a graph of K launches of that call alone (events between
+    kernels inside one graph would add their own gaps). Then each call is
+    timed alone with CUDA events (eager launches, so the interval includes
+    the launch), after writing the 512 MB `flush` buffer so that no call
+    finds its inputs in L2 (p10 / p50 / p90); steps smaller than the flush
+    are also timed L2-hot, calls back to back on one set."""
+    barrier = barrier or (lambda: None)
+    rank_max = rank_max or (lambda x: x)
+    n = len(paths)
+    wl = paths[0].wl
+    with nvtx(f"{wl.name}: warm-up"):
+        for _ in range(warmup):
+            for p in paths:
+                p.step()
+        torch.cuda.synchronize()
+    for p in paths:
+        st = int(p.status[0].item())
+        if st:
+            raise RuntimeError(f"device status after warm-up: {st}")
+    bts = [step_bytes(p, backward) for p in paths]
+    b_total = sum(bts[i % n]["step"] for i in range(K))
+
+    graph = capture(lambda i: paths[i % n].step(), K)
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with nvtx(f"{wl.name}: timed steps"), ClockSampler(device_index) as clk:
+        start.record()
+        graph.replay()
+        stop.record()
+        torch.cuda.synchronize()
+    barrier()
+    del graph
+    ms = rank_max(start.elapsed_time(stop))
+
+    calls = ["layout_dispatch", "combine"]
+    if kernels:
+        calls += ["layout", "dispatch"]
+    if wl.B:
+        calls.append("plan_prefetch")
+    if backward:
+        calls += ["combine_backward", "dispatch_backward"]
+        if wl.B:
+            calls.append("reduce_slot_grads")
+    avg = {}
+    with nvtx(f"{wl.name}: per-call graphs"):
+        for name in calls:
+            g = capture(lambda i: getattr(paths[i % n], name)(), K)
+            avg[name] = replay_ms(g) / K * 1e3     # us per launch
+            del g
+    per_call = {}
+    timed = ["layout_dispatch", "combine"] + (["plan_prefetch"] if wl.B else [])
+    # l2_flushed: 512 MB written before each call, so L2 holds none of the
+    # call's data but is full of dirty lines the call's own traffic must
+    # write back first; l2_clean: the same write, then a read of the 512 MB,
+    # so L2 holds none of the call's data and only clean lines
+    modes = [("l2_flushed", "write"), ("l2_clean", "write+read")]
+    if bts[0]["step"] < flush.numel():
+        modes.append(("l2_hot", None))
+    flush64 = flush.view(torch.int64)
+    with nvtx(f"{wl.name}: per-call distribution"):
+        for mode, how in modes:
+            for name in timed:
+                n_calls = 10 if name == "plan_prefetch" else 50
+                evs = []
+                if how is None:
+                    # keep the GPU busy while the host enqueues the calls,
+                    # so that they run back to back and each interval is
+                    # GPU time
+                    torch.cuda._sleep(4_000_000)
+                for c in range(n_calls):
+                    p = paths[c % n] if how else paths[0]
+                    if how:
+                        flush.fill_(1)
+                    if how == "write+read":
+                        flush64.max()
+                    a_, b_ = (torch.cuda.Event(enable_timing=True),
+                              torch.cuda.Event(enable_timing=True))
+                    a_.record()
+                    getattr(p, name)()
+                    b_.record()
+                    evs.append((a_, b_))
+                torch.cuda.synchronize()
+                us = np.array([a_.elapsed_time(b_) * 1e3 for a_, b_ in evs])
+                per_call.setdefault(mode, {})[name] = percentiles(us)
+    for p in paths:
+        st = int(p.status[0].item())
+        if st:
+            raise RuntimeError(f"device status after timing: {st}")
+    # bytes per call averaged over the sets
+    mean_b = {k: sum(b[k] for b in bts) / n for k in bts[0]}
+    return {"ms": ms, "K": K, "bytes_total": b_total, "bytes": mean_b,
+            "avg_us": avg, "per_call_us": per_call, "clocks": clk.summary(),
+            "sets": n}
+
+
+def gbps(nbytes, us):
+    return nbytes / (us * 1e-6) / 1e9 if us > 0 else None
+
+
+def kernel_names(wl, sms=148):
+    """Kernels the step launches, by the library's size rules (mirrored
+    here; tests/test_bench_accounting.py pins the mirror)."""
+    one_launch = layout_dispatch_kernels(wl, sms) == 1
+    prec = "fp8" if wl.fp8 else "bf16"
+    if one_launch:
+        disp = f"k_layout_small<{prec}>"
+    else:
+        disp = f"k_dispatch_{prec}"
+    return {"one_launch": one_launch, "dispatch": disp,
+            "combine": combine_kernel(wl, sms)}
+
+
+def arithmetic(wl):
+    return (("fp8-e4m3 dispatch (1x128 fp32 scales, x/scale in fp32)"
+             if wl.fp8 else "bf16 dispatch (bit copy)") +
+            ", bf16 combine with fp32 fma accumulation")
+
+
+def workload_summary(wl, m, peak):
+    """The line for a workload other than the headline one."""
+    avg, b = m["avg_us"], m["bytes"]
+    names = kernel_names(wl)
+    out = {
+        "workload": wl.describe,
+        "arithmetic": arithmetic(wl),
+        "input_sets": m["sets"],
+        "l2": (f"{m['sets']} input sets rotated, {m['sets']} x "
+               f"{b['step'] / 1e6:.0f} MB per rotation > the 126 MB L2"
+               if m["sets"] > 1 else
+               f"one input set; every step moves {b['step'] / 1e6:.0f} MB, "
+               "more than the 126 MB L2"),
+        "step_us": round(m["ms"] / m["K"] * 1e3, 2),
+        "step_GBps": round(m["bytes_total"] / (m["ms"] * 1e-3) / 1e9, 1),
+        "graph_us": {k: round(v, 2) for k, v in avg.items()},
+        "per_call_us": m["per_call_us"],
+        "kernels": names,
+        "clocks": m["clocks"],
+    }
+    rates = {}
+    for k in ("layout_dispatch", "combine", "plan_prefetch"):
+        if k in avg and b[k]:
+            r = gbps(b[k], avg[k])
+            rates[k] = {"bytes": int(b[k]), "GBps": round(r, 1),
+                        "frac_of_measured": round(r / peak, 4),
+                        "frac_of_8TBps": round(r / NOMINAL_HBM_GBS, 4)}
+            fl = m["per_call_us"].get("l2_flushed", {}).get(k)
+            if fl:
+                r50 = gbps(b[k], fl["p50"])
+                rates[k]["flushed_p50_GBps"] = round(r50, 1)
+                rates[k]["flushed_p50_frac_of_measured"] = round(r50 / peak, 4)
+    out["rates"] = rates
+    return out
+
+
+def time_epbuffer(path, K, dev):
+    """One pass of the pages' Buffer call shape (EPBuffer.dispatch, then
+    EPBuffer.combine on stand-in expert outputs), timed beside the raw-call
+    step: a graph of K passes, and K eager passes with the Python of the
+    binding and of EPBuffer on the host side."""
+    from combine_ep_layout_09_b200 import EPBuffer
+    wl = path.wl
+    buf = EPBuffer(wl.S, wl.H, wl.K, wl.E, wl.R, token_padding=wl.pad,
+                   fp8=wl.fp8, device=dev)
+
+    def one(_i=0):
+        _, _, _, h = buf.dispatch(path.hidden, path.w, path.topk)
+        buf.combine(h, path.y)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    g = capture(one, K)
+    graph_us = replay_ms(g) / K * 1e3
+    del g
+    a_, b_ = (torch.cuda.Event(enable_timing=True),
+              torch.cuda.Event(enable_timing=True))
+    a_.record()
+    for _ in range(K):
+        one()
+    b_.record()
+    torch.cuda.synchronize()
+    eager_us = a_.elapsed_time(b_) / K * 1e3
+    buf.check()
+    del buf
+    return {"graph_us_per_pass": round(graph_us, 2),
+            "eager_us_per_pass": round(eager_us, 2),
+            "calls": "EPBuffer.dispatch (ep_layout_dispatch) + "
+                     "EPBuffer.combine (ep_combine_recv_weights: receive-"
+                     "side weights, gathered weights written, no allocation)",
+            "launches_per_pass": layout_dispatch_kernels(wl) + 1}
+
+
+EXTRA_WORKLOADS = {"decode": 4, "skewed": 1, "balanced": 1}
+
+
 def run_gpu(args, wl):
     ws, rank, local = dist_info()
     torch.cuda.set_device(local)
@@ -398,154 +686,66 @@ def run_gpu(args, wl):
     def rank_max(x: float) -> float:
         return max_over_ranks(x, dev)
 
+    K = args.steps
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    # the headline workload: one input set (every step moves more than L2)
+    # unless the step is smaller than the 512 MB flush, then four
+    n_sets = 1
     path = Path(wl, dev, seed_offset=rank)
     if args.backward:
         path.enable_backward(seed_offset=rank)
+    paths = [path]
     torch.cuda.synchronize()
-    # warm-up (also settles the used-row count for byte accounting)
-    for _ in range(args.warmup):
-        path.step()
+    path.step()
     torch.cuda.synchronize()
-    st = int(path.status[0].item())
-    if st:
-        raise RuntimeError(f"device status after warm-up: {st}")
-    used = int(path.offsets[-1].item())
-    n_slots = int((path.plan["slot"] >= 0).sum().item()) if wl.B else 0
-
-    b_lay = bytes_layout(wl.N, wl.K, wl.E, used)
-    b_dis = bytes_dispatch(wl.N, wl.K, wl.H, wl.fp8, used)
-    b_com = bytes_combine(wl.N, wl.K, wl.H)
-    b_pre = bytes_prefetch(n_slots, wl.H, wl.I) if wl.B else 0
-    b_cbw = bytes_combine_backward(wl.N, wl.K, wl.H, used) if args.backward else 0
-    b_dbw = bytes_dispatch_backward(wl.N, wl.K, wl.H) if args.backward else 0
-    b_red = (bytes_reduce_slot_grads(path.plan["slot"].cpu().numpy(), wl.H,
-                                     wl.I) if args.backward and wl.B else 0)
-    b_step = b_lay + b_dis + b_com + b_pre + b_cbw + b_dbw + b_red
-
-    # The K timed steps are captured once into a CUDA graph (the library is
-    # capture-safe: no allocation, no synchronisation) and replayed once, so
-    # no host launch gap sits between kernels. Each kernel's own average is
-    # then timed the same way, from a graph of K launches of that kernel
-    # alone (events between kernels inside one graph would add their own
-    # gaps to the kernels they bracket).
-    K = args.steps
-
-    def capture(fn, n):
-        cs = torch.cuda.Stream()
-        cs.wait_stream(torch.cuda.current_stream())
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=cs):
-            for _ in range(n):
-                fn()
-        torch.cuda.synchronize()
-        return g
-
-    def replay_ms(g):
-        a_, b_ = (torch.cuda.Event(enable_timing=True),
-                  torch.cuda.Event(enable_timing=True))
-        a_.record()
-        g.replay()
-        b_.record()
-        torch.cuda.synchronize()
-        return a_.elapsed_time(b_)
-
-    graph = capture(path.step, K)
-    start = torch.cuda.Event(enable_timing=True)
-    stop = torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        start.record()
-        graph.replay()
-        stop.record()
-        torch.cuda.synchronize()
-    barrier()
-    del graph
-    parts = {"layout_dispatch": path.layout_dispatch, "layout": path.layout,
-             "dispatch": path.dispatch, "combine": path.combine}
-    if wl.B > 0:
-        parts["plan_prefetch"] = path.plan_prefetch
-    if args.backward:
-        parts["combine_backward"] = path.combine_backward
-        parts["dispatch_backward"] = path.dispatch_backward
-        if wl.B > 0:
-            parts["reduce_slot_grads"] = path.reduce_slot_grads
-    avg = {"plan_prefetch": 0.0, "combine_backward": 0.0,
-           "dispatch_backward": 0.0, "reduce_slot_grads": 0.0}
-    for name, fn in parts.items():
-        g = capture(fn, K)
-        avg[name] = replay_ms(g) / K * 1e3     # us per launch
-        del g
-    med = avg
-    # Per-call distribution: each call timed alone with CUDA events (eager
-    # launches, so the interval includes the launch), after writing a 512 MB
-    # scratch buffer (4x the L2) so that no call finds its inputs in L2; the
-    # small decode batch is also timed L2-hot, calls back to back.
-    per_call = {}
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
-    calls = {"layout_dispatch": path.layout_dispatch, "combine": path.combine}
-    if wl.B > 0:
-        calls["plan_prefetch"] = path.plan_prefetch
-    modes = [("l2_flushed", True)] + ([("l2_hot", False)]
-                                      if b_step < 512e6 else [])
-    for mode, do_flush in modes:
-        for name, fn in calls.items():
-            n_calls = 10 if name == "plan_prefetch" else 50
-            evs = []
-            if not do_flush:
-                # keep the GPU busy while the host enqueues the calls, so
-                # that they run back to back and each interval is GPU time
-                torch.cuda._sleep(4_000_000)
-            for _ in range(n_calls):
-                if do_flush:
-                    flush.fill_(1)
-                a_, b_ = (torch.cuda.Event(enable_timing=True),
-                          torch.cuda.Event(enable_timing=True))
-                a_.record()
-                fn()
-                b_.record()
-                evs.append((a_, b_))
-            torch.cuda.synchronize()
-            us = np.array([a_.elapsed_time(b_) * 1e3 for a_, b_ in evs])
-            per_call.setdefault(mode, {})[name] = {
-                "p10": round(float(np.percentile(us, 10)), 2),
-                "p50": round(float(np.percentile(us, 50)), 2),
-                "p90": round(float(np.percentile(us, 90)), 2),
-                "calls": n_calls}
-    del flush
-    ms = start.elapsed_time(stop)
-    ms_max = rank_max(ms)
-    st = int(path.status[0].item())
-    if st:
-        raise RuntimeError(f"device status after timing: {st}")
+    if step_bytes(path, args.backward)["step"] < flush.numel():
+        n_sets = 4
+        for j in range(1, n_sets):
+            p = Path(wl, dev, seed_offset=rank + 100 * j)
+            if args.backward:
+                p.enable_backward(seed_offset=rank + 100 * j)
+            paths.append(p)
+    m = measure(paths, K, args.warmup, args.backward, local, flush, barrier,
+                rank_max)
+    avg, b = m["avg_us"], m["bytes"]
+    ms_max = m["ms"]
 
     # ---- end to end: host buffers in, host result out, every step -------
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, path, b_step, rank_max, barrier)
+        with nvtx(f"{wl.name}: end to end"):
+            e2e = run_e2e(args, path, b["step"], rank_max, barrier)
+
+    epbuf = None
+    if ws == 1 and not args.no_epbuffer:
+        with nvtx(f"{wl.name}: EPBuffer pass"):
+            epbuf = time_epbuffer(path, K, dev)
 
     result = None
     if rank == 0:
         peak, peak_src = measured_peak()
-        value = total_value_gbs(b_step, K, ws, ms_max)
-        comb_gbs = b_com / (avg["combine"] * 1e-6) / 1e9
-        dis_gbs = b_dis / (avg["dispatch"] * 1e-6) / 1e9
-        ld_gbs = (b_lay + b_dis) / (avg["layout_dispatch"] * 1e-6) / 1e9
-        one_launch = layout_dispatch_kernels(wl) == 1
+        value = total_value_gbs(m["bytes_total"] / K, K, ws, ms_max)
+        names = kernel_names(wl)
+        one_launch = names["one_launch"]
+        comb_gbs = gbps(b["combine"], avg["combine"])
+        dis_gbs = gbps(b["dispatch"], avg["dispatch"])
+        ld_gbs = gbps(b["layout_dispatch"], avg["layout_dispatch"])
         # the dominant kernel: combine, or the dispatch side's longest kernel
         # (the single layout+dispatch kernel of a small batch)
         if one_launch:
-            cand = ("layout_dispatch", "k_layout_small", "layout_small.cu",
-                    b_lay + b_dis, ld_gbs)
+            cand = ("layout_dispatch", names["dispatch"], "layout_small.cu",
+                    b["layout_dispatch"], ld_gbs)
         else:
-            cand = ("dispatch", "k_dispatch", "dispatch.cu", b_dis, dis_gbs)
+            cand = ("dispatch", names["dispatch"], "dispatch.cu",
+                    b["dispatch"], dis_gbs)
         if avg["combine"] >= avg[cand[0]]:
-            cand = ("combine", "k_combine", "combine.cu", b_com, comb_gbs)
+            cand = ("combine", names["combine"], "combine.cu", b["combine"],
+                    comb_gbs)
         dom, kname, ksrc, dom_bytes, dom_gbs = cand
-        kern = (kname, ksrc)
-        src = os.path.join(ROOT, "combine_ep_layout_09_b200", "csrc", kern[1])
-        traffic = traffic_from_profiles(kern[0], wl.name, src)
-        clocks = clk.summary()
+        src = os.path.join(ROOT, "combine_ep_layout_09_b200", "csrc", ksrc)
+        traffic = traffic_from_profiles(kname, wl.name, src)
+        clocks = m["clocks"]
+        per_call = m["per_call_us"]
         result = {
             "metric": METRIC,
             "value": round(value, 1),
@@ -557,10 +757,12 @@ def run_gpu(args, wl):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "f32",
+            "dtype": ("e4m3+bf16, fp32 accumulate" if wl.fp8 else
+                      "bf16, fp32 accumulate"),
             "data": "synthetic",
             "config": {
                 "workload": wl.describe,
+                "arithmetic": arithmetic(wl),
                 "step": ("ep_layout_dispatch (" +
                          ("one launch" if one_launch else
                           "ep_layout + ep_dispatch") + ") + " +
@@ -570,47 +772,54 @@ def run_gpu(args, wl):
                           if args.backward else "") +
                          (" + ep_reduce_slot_grads"
                           if args.backward and wl.B else "")),
-                "bytes_per_step": b_step,
-                "used_rows": used,
-                "l2": (f"no flush: every step moves {b_step / 1e6:.0f} MB,"
-                       " more than the 126 MB L2" if b_step > 126e6 else
-                       "L2-resident: the step moves less than the 126 MB "
-                       "L2"),
+                "bytes_per_step": int(b["step"]),
+                "used_rows": int(b["used_rows"]),
+                "input_sets": m["sets"],
+                "l2": (f"no flush: every step moves {b['step'] / 1e6:.0f} MB,"
+                       " more than the 126 MB L2" if m["sets"] == 1 else
+                       f"{m['sets']} input sets rotated, "
+                       f"{m['sets'] * b['step'] / 1e6:.0f} MB per rotation, "
+                       "more than the 126 MB L2"),
                 "parallelism": f"{ws} independent replica(s), one per GPU",
                 "timing": "K steps captured in one CUDA graph, replayed "
-                          "once, CUDA events around the replay; per-kernel "
-                          "times from a graph of K launches of that kernel",
+                          "once, CUDA events around the replay; per-call "
+                          "averages from a graph of K launches of that call",
             },
             "per_call_us": per_call,
             "breakdown": {
-                "layout_dispatch_us": round(med["layout_dispatch"], 2),
+                "layout_dispatch_us": round(avg["layout_dispatch"], 2),
                 "layout_dispatch_GBps": round(ld_gbs, 1),
                 "layout_dispatch_one_launch": one_launch,
-                "layout_us": round(med["layout"], 2),
-                "dispatch_us": round(med["dispatch"], 2),
-                "combine_us": round(med["combine"], 2),
-                "plan_prefetch_us": round(med["plan_prefetch"], 2),
-                "layout_plus_dispatch_us": round(med["layout"] +
-                                                 med["dispatch"], 2),
+                "layout_us": round(avg["layout"], 2),
+                "dispatch_us": round(avg["dispatch"], 2),
+                "combine_us": round(avg["combine"], 2),
+                "plan_prefetch_us": round(avg.get("plan_prefetch", 0.0), 2),
+                "layout_plus_dispatch_us": round(avg["layout"] +
+                                                 avg["dispatch"], 2),
                 "dispatch_GBps": round(dis_gbs, 1),
                 "combine_GBps": round(comb_gbs, 1),
                 "dispatch_payload_GBps": round(
                     payload_dispatch(wl.N, wl.K, wl.H, wl.fp8) /
                     (avg["dispatch"] * 1e-6) / 1e9, 1),
-                "combine_backward_us": round(med["combine_backward"], 2),
-                "dispatch_backward_us": round(med["dispatch_backward"], 2),
-                "combine_backward_GBps": round(
-                    b_cbw / (avg["combine_backward"] * 1e-6) / 1e9, 1)
+                "combine_backward_us": round(avg.get("combine_backward", 0), 2),
+                "dispatch_backward_us": round(avg.get("dispatch_backward", 0),
+                                              2),
+                "combine_backward_GBps": round(gbps(
+                    b["combine_backward"], avg["combine_backward"]), 1)
                 if args.backward else None,
-                "dispatch_backward_GBps": round(
-                    b_dbw / (avg["dispatch_backward"] * 1e-6) / 1e9, 1)
+                "dispatch_backward_GBps": round(gbps(
+                    b["dispatch_backward"], avg["dispatch_backward"]), 1)
                 if args.backward else None,
-                "reduce_slot_grads_us": round(med["reduce_slot_grads"], 2),
-                "reduce_slot_grads_GBps": round(
-                    b_red / (avg["reduce_slot_grads"] * 1e-6) / 1e9, 1)
-                if b_red else None,
-                "dispatch_bytes": b_dis, "combine_bytes": b_com,
-                "layout_bytes": b_lay, "prefetch_bytes": b_pre,
+                "reduce_slot_grads_us": round(avg.get("reduce_slot_grads", 0),
+                                              2),
+                "reduce_slot_grads_GBps": round(gbps(
+                    b["reduce_slot_grads"], avg["reduce_slot_grads"]), 1)
+                if b["reduce_slot_grads"] else None,
+                "dispatch_bytes": int(b["dispatch"]),
+                "combine_bytes": int(b["combine"]),
+                "layout_bytes": int(b["layout"]),
+                "prefetch_bytes": int(b["plan_prefetch"]),
+                "kernels": names,
                 "frac_of_8TBps": {
                     "dispatch": round(dis_gbs / NOMINAL_HBM_GBS, 4),
                     "layout_dispatch": round(ld_gbs / NOMINAL_HBM_GBS, 4),
@@ -622,24 +831,47 @@ def run_gpu(args, wl):
             },
             "roofline": {
                 "bound": "hbm",
-                "kernel": kern[0],
+                "kernel": kname,
+                "call": dom,
                 "achieved": round(dom_gbs, 1),
                 "peak": peak,
                 "unit": "GB/s",
                 "frac": round(dom_gbs / peak, 4),
                 "traffic": traffic,
-                "algorithmic_bytes": dom_bytes,
+                "algorithmic_bytes": int(dom_bytes),
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_src == "measured" else "fallback 6.65 TB/s",
             },
             "clocks": clocks,
             "e2e": e2e,
+            "epbuffer": epbuf,
             "gpu_launches": path.launches_per_step * K,
             "gpu_launches_note": "kernels of libeplayout.so in the timed "
                                  "region" + ("" if one_launch else
                                              "; ep_layout adds one "
                                              "cudaMemsetAsync per step"),
         }
+    del paths, path
+    torch.cuda.empty_cache()
+
+    # ---- the other workloads, in the same process (one GPU only) --------
+    extras = {}
+    if ws == 1 and not args.no_extra_workloads and wl.name == "prefill" \
+            and args.tokens_per_rank is None:
+        peak, _ = measured_peak()
+        for name, sets in EXTRA_WORKLOADS.items():
+            xw = workloads.WORKLOADS[name]
+            with nvtx(f"{name}: setup"):
+                xp = [Path(xw, dev, seed_offset=100 * j) for j in range(sets)]
+                torch.cuda.synchronize()
+            xm = measure(xp, K, args.warmup, False, local, flush,
+                         kernels=False)
+            extras[name] = workload_summary(xw, xm, peak)
+            del xp
+            torch.cuda.empty_cache()
+    if result is not None and extras:
+        result["workloads"] = extras
+    del flush
     if ws > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -851,6 +1083,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-epbuffer", action="store_true",
+                    help="skip timing the EPBuffer pass")
+    ap.add_argument("--no-extra-workloads", action="store_true",
+                    help="time only the selected workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--backward", action="store_true",
                     help="add the backward pair to the step")

@@ -69,17 +69,21 @@ __device__ __forceinline__ float entry_weight(const Weights& wt, int64_t t,
 }
 
 // KT > 0: K known at compile time; KT == 0: runtime K, in chunks of kChunk
-// terms (the chunks run in k order, so the fma order is unchanged).
-template <int KT>
-__global__ void __launch_bounds__(kCombineMaxThreads)
+// terms (the chunks run in k order, so the fma order is unchanged). kRows:
+// weights per receive row (wts.rows), else per entry or unit (wts.tok).
+// Two CTAs per SM: at most 64 registers a thread.
+template <int KT, bool kRows>
+__global__ void __launch_bounds__(kCombineMaxThreads, 2)
     k_combine(const uint16_t* __restrict__ y, const int32_t* __restrict__ pos,
               Weights wts, int64_t N, int Kr, int H, int64_t cap,
               uint16_t* __restrict__ out, int32_t* __restrict__ status) {
   const int K = KT > 0 ? KT : Kr;
   const int V = H >> 3;
+  if constexpr (kRows) wts.tok = nullptr;
+  else wts.rows = nullptr;
   for (int64_t t = blockIdx.x; t < N; t += gridDim.x) {
     const int32_t* pt = pos + t * K;
-    if (wts.rows && wts.gathered && threadIdx.x < K) {
+    if (kRows && wts.gathered && threadIdx.x < K) {
       const int32_t p = __ldg(pt + threadIdx.x);
       wts.gathered[t * K + threadIdx.x] = entry_weight(wts, t, K, threadIdx.x, p, cap);
     }
@@ -246,12 +250,13 @@ __global__ void __launch_bounds__((kTmaMaxConsumerWarps + 1) * 32, 1)
       }
       // Every lane's weight is in shared memory before lane 0 arrives: the
       // arrive (a release) then covers the whole warp's writes, and the
-      // consumers' wait on the phase (an acquire) sees them.
+      // consumers' wait on the phase (an acquire) sees them. The loads may
+      // be issued before lane 0's arrive lands: the phase needs that arrive
+      // as well as the bytes, whatever their order.
       wk[s * 32 + lane] = wv;
       if (lane == 0) vmask[s] = m;
       __syncwarp();
       if (lane == 0) mbar_arrive_expect_tx(&full[s], uint32_t(__popc(m)) * bytes);
-      __syncwarp();
       if (valid)
         bulk_g2s(in_base + size_t(s) * sh.in_bytes + size_t(lane) * sh.part_ch * 2,
                  y + int64_t(p) * H + c0, bytes, &full[s]);
@@ -323,10 +328,10 @@ cudaError_t run_tma(const uint16_t* y, const int32_t* pos, const Weights& w,
   return cudaGetLastError();
 }
 
-template <int KT>
-cudaError_t run(const uint16_t* y, const int32_t* pos, const Weights& w,
-                int64_t N, int K, int H, int64_t cap, uint16_t* out,
-                int num_sms, int32_t* status, cudaStream_t stream) {
+template <int KT, bool kRows>
+cudaError_t run_k(const uint16_t* y, const int32_t* pos, const Weights& w,
+                  int64_t N, int K, int H, int64_t cap, uint16_t* out,
+                  int num_sms, int32_t* status, cudaStream_t stream) {
   const int V = H >> 3;
   // Threads per CTA: the fewest passes over the row with <= 512 threads.
   const int passes = (V + kCombineMaxThreads - 1) / kCombineMaxThreads;
@@ -334,14 +339,23 @@ cudaError_t run(const uint16_t* y, const int32_t* pos, const Weights& w,
   threads = std::max(32, (threads + 31) / 32 * 32);
   int per_sm = 0;
   cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-      &per_sm, k_combine<KT>, threads, 0);
+      &per_sm, k_combine<KT, kRows>, threads, 0);
   if (err != cudaSuccess) return err;
   per_sm = std::max(1, per_sm);
   const int64_t grid =
       std::max<int64_t>(1, std::min<int64_t>(N, int64_t(num_sms) * per_sm));
-  k_combine<KT><<<int(grid), threads, 0, stream>>>(y, pos, w, N, K, H, cap,
-                                                   out, status);
+  k_combine<KT, kRows><<<int(grid), threads, 0, stream>>>(y, pos, w, N, K, H,
+                                                          cap, out, status);
   return cudaGetLastError();
+}
+
+template <int KT>
+cudaError_t run(const uint16_t* y, const int32_t* pos, const Weights& w,
+                int64_t N, int K, int H, int64_t cap, uint16_t* out,
+                int num_sms, int32_t* status, cudaStream_t stream) {
+  if (w.rows)
+    return run_k<KT, true>(y, pos, w, N, K, H, cap, out, num_sms, status, stream);
+  return run_k<KT, false>(y, pos, w, N, K, H, cap, out, num_sms, status, stream);
 }
 
 }  // namespace

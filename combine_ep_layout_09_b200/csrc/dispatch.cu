@@ -173,7 +173,10 @@ __global__ void __launch_bounds__(32)
 // fp8: producer warp + consumer warps, output stage bulk-stored K times
 // ---------------------------------------------------------------------------
 
-__global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32)
+// Two CTAs share an SM (their stages take ~100 KB each), so a thread may
+// use at most 60 registers: with 15 warps per CTA anything above 64 rounds
+// to 72 per thread and leaves room for one CTA only.
+__global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 2)
     k_dispatch_fp8(const uint16_t* __restrict__ hidden,
                    const float* __restrict__ w, const int32_t* __restrict__ pos,
                    const int32_t* __restrict__ row_src,

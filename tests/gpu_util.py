@@ -157,3 +157,29 @@ def gpu_layout_dispatch(topk: np.ndarray, hidden_dev: torch.Tensor,
                 pos=pos[:N].cpu().numpy(), row_src=row_src[:cap].cpu().numpy(),
                 recv=recv, scales=scales, recv_w=recv_w,
                 status=int(st[0].item()), cap=cap)
+
+
+ROW_CHUNK = 16384     # receive rows per device -> host copy
+
+
+def host_rows(t: torch.Tensor, lo: int, hi: int) -> np.ndarray:
+    """Rows [lo, hi) of a device tensor as host numpy bit patterns."""
+    part = t[lo:hi]
+    if part.dtype == torch.bfloat16:
+        return u16(part)
+    if part.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return part.view(torch.uint8).cpu().numpy()
+    return part.cpu().numpy()
+
+
+def assert_rows_equal(dev: torch.Tensor, ref: np.ndarray, what: str):
+    """Every row of a device tensor equal to `ref`, compared in chunks of
+    ROW_CHUNK rows so that the host holds one chunk of the device data."""
+    assert dev.shape[0] == ref.shape[0], what
+    for lo in range(0, ref.shape[0], ROW_CHUNK):
+        hi = min(lo + ROW_CHUNK, ref.shape[0])
+        got = host_rows(dev, lo, hi)
+        if not np.array_equal(got, ref[lo:hi]):
+            bad = np.nonzero((got != ref[lo:hi]).reshape(hi - lo, -1).any(1))[0]
+            raise AssertionError(f"{what}: {len(bad)} rows differ in "
+                                 f"[{lo}, {hi}), first {lo + int(bad[0])}")

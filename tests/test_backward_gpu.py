@@ -9,8 +9,9 @@ import torch
 import combine_ep_layout_09_b200 as ep
 import oracle
 import workloads
-from gpu_util import (DEV, RECV_BF16_FILL, gpu_layout, rows_to_host,
-                      status_tensor, to_bf16_dev, to_dev, u16)
+from gpu_util import (DEV, RECV_BF16_FILL, assert_rows_equal, gpu_layout,
+                      host_rows, rows_to_host, status_tensor, to_bf16_dev,
+                      to_dev, u16)
 
 pytestmark = pytest.mark.gpu
 
@@ -85,28 +86,38 @@ def test_combine_backward_small(R, S, K, E, H, pad):
     assert np.all(np.abs(got - ref_w) <= 1e-2 * np.abs(ref_w).max() + 1e-6)
 
 
-def test_combine_backward_full_size_sampled():
-    wl = workloads.WORKLOADS["skewed"]
+@pytest.mark.parametrize("name", ["skewed", "prefill"])
+def test_backward_full_size(name):
+    # every row of the expert-output gradient (padding rows included) and
+    # every token's route-weight gradient and token gradient, at full size
+    wl = workloads.WORKLOADS[name]
     topk, w = workloads.routing(wl)
     lay, cap, y, g, rows, gw = run_combine_backward(topk, w, wl.R, wl.S, wl.E,
                                                      wl.H, wl.pad, 9)
     o = oracle.layout(topk, wl.E, wl.pad, cap)
-    rng = np.random.default_rng(3)
-    toks = np.sort(rng.choice(wl.N, 256, replace=False))
-    g_s = rows_to_host(g, toks)
-    r = o["pos"][toks]
-    got_rows = rows_to_host(rows, r.ravel()).reshape(len(toks), wl.K, wl.H)
-    for k in range(wl.K):
-        prod = (as_f32(g_s) * w[toks, k:k + 1]).astype(np.float32)
-        ref = torch.from_numpy(prod).to(torch.bfloat16).view(
-            torch.int16).numpy().view(np.uint16)
-        np.testing.assert_array_equal(got_rows[:, k], ref)
-    y_rows = rows_to_host(y, r.ravel())
-    weight_grad_ok(gw.cpu().numpy()[toks].astype(np.float64), g_s, y_rows,
-                   wl.K, wl.H)
-    used = int(o["offsets"][-1])
-    pad_rows = np.where(o["row_src"][:used] < 0)[0][:500]
-    assert np.all(rows_to_host(rows, pad_rows) == 0)
+    g_host = u16(g)
+    ref_rows = oracle.combine_backward_rows(g_host, w, o, wl.E, cap,
+                                            fill=RECV_BF16_FILL)
+    assert_rows_equal(rows, ref_rows, "grad rows")
+    del ref_rows
+    gx = torch.empty(wl.N, wl.H, dtype=torch.bfloat16, device=DEV)
+    st = status_tensor()
+    ep.ep_dispatch_backward(rows, lay["dev"]["pos"], wl.N, wl.K, wl.H, gx,
+                            status=st)
+    torch.cuda.synchronize()
+    assert int(st[0].item()) == 0
+    gw_host = gw.cpu().numpy()
+    chunk = 2048
+    for t0 in range(0, wl.N, chunk):
+        t1 = min(wl.N, t0 + chunk)
+        r = o["pos"][t0:t1].ravel()
+        local = np.arange(len(r), dtype=np.int32).reshape(t1 - t0, wl.K)
+        y_rows = rows_to_host(y, r)
+        weight_grad_ok(gw_host[t0:t1].astype(np.float64), g_host[t0:t1],
+                       y_rows, wl.K, wl.H)
+        gr_rows = rows_to_host(rows, r)
+        np.testing.assert_array_equal(host_rows(gx, t0, t1),
+                                      oracle.dispatch_backward(gr_rows, local))
 
 
 def test_gather_route_weights():

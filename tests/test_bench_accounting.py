@@ -59,3 +59,27 @@ def test_launch_count_follows_the_library_rule(S, K, expect):
     assert (limit, per_cta) == (32768, 1024)   # the numbers bench.py mirrors
     wl = workloads.scaled(workloads.WORKLOADS["prefill"], S=S, K=K)
     assert bench.layout_dispatch_kernels(wl) == expect
+
+
+def _combine_constants():
+    src = open(os.path.join(ROOT, "combine_ep_layout_09_b200", "csrc",
+                            "combine.cu")).read()
+    stage = re.search(r"kTmaStageTarget\s*=\s*(\d+)\s*\*\s*1024", src)
+    rule = re.search(r"sh\.smem\s*<=\s*(\d+)\s*\*\s*1024\s*&&\s*N\s*\*\s*"
+                     r"sh\.parts\s*>=\s*(\d+)\s*\*", src)
+    assert stage and rule
+    return int(stage.group(1)), int(rule.group(1)), int(rule.group(2))
+
+
+@pytest.mark.parametrize("N,K,H,expect", [
+    (32768, 8, 7168, "k_combine_tma"),    # prefill: 2 parts per row
+    (1024, 8, 7168, "k_combine<8>"),      # decode: 2048 units < 16 per SM
+    (2500, 8, 1024, "k_combine_tma"),     # one part, 2500 units
+    (300, 8, 7168, "k_combine<8>"),
+    (100000, 1, 32768, "k_combine<1>"),   # 64 KB parts: stages above 200 KB
+])
+def test_combine_kernel_follows_the_library_rule(N, K, H, expect):
+    assert _combine_constants() == (64, 200, 16)   # what bench.py mirrors
+    wl = workloads.scaled(workloads.WORKLOADS["prefill"], S=N // 8, K=K, H=H)
+    wl = workloads.scaled(wl, R=1, S=N)
+    assert bench.combine_kernel(wl) == expect

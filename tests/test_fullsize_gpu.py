@@ -29,32 +29,12 @@ import bench
 import oracle
 import workloads
 from gpu_util import (DEV, RECV_BF16_FILL, RECV_FP8_FILL, RECV_W_FILL,
-                      ROW_SRC_FILL, SCALE_FILL, rows_to_host, u16)
+                      ROW_SRC_FILL, SCALE_FILL, assert_rows_equal, host_rows,
+                      rows_to_host, u16)
 
 pytestmark = pytest.mark.gpu
 
-ROW_CHUNK = 16384     # receive rows per device -> host copy
 TOKEN_CHUNK = 2048    # tokens per combine comparison
-
-
-def host_rows(t: torch.Tensor, lo: int, hi: int) -> np.ndarray:
-    part = t[lo:hi]
-    if part.dtype == torch.bfloat16:
-        return u16(part)
-    if part.dtype in (torch.uint8, torch.float8_e4m3fn):
-        return part.view(torch.uint8).cpu().numpy()
-    return part.cpu().numpy()
-
-
-def assert_rows_equal(dev: torch.Tensor, ref: np.ndarray, what: str):
-    assert dev.shape[0] == ref.shape[0], what
-    for lo in range(0, ref.shape[0], ROW_CHUNK):
-        hi = min(lo + ROW_CHUNK, ref.shape[0])
-        got = host_rows(dev, lo, hi)
-        if not np.array_equal(got, ref[lo:hi]):
-            bad = np.nonzero((got != ref[lo:hi]).reshape(hi - lo, -1).any(1))[0]
-            raise AssertionError(f"{what}: {len(bad)} rows differ in "
-                                 f"[{lo}, {hi}), first {lo + int(bad[0])}")
 
 
 def row_checksums(W: torch.Tensor) -> torch.Tensor:
