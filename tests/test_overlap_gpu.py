@@ -20,7 +20,7 @@ def test_dispatch_and_combine_beside_a_gemm(fp8):
                           fp8=fp8)
     topk, w = workloads.routing(wl)
     hid = workloads.hidden_states(wl, device=DEV)
-    buf = ep.EPBuffer(wl.S, wl.H, wl.K, wl.E, wl.R, num_sms=64, fp8=fp8,
+    buf = ep.EPBuffer(wl.S, wl.H, wl.K, wl.E, wl.R, num_sms=74, fp8=fp8,
                       device=DEV)
     a = torch.randn(4096, 4096, device=DEV, dtype=torch.bfloat16)
     y = workloads.expert_outputs(buf.cap, wl.H, 5, device=DEV)
@@ -34,7 +34,10 @@ def test_dispatch_and_combine_beside_a_gemm(fp8):
         out, _ = buf.combine(hd, y)
     torch.cuda.synchronize()
     buf.check()
-    assert torch.isfinite(c.float()).all()
+    # the GEMM that ran beside them gives what it gives alone
+    c_alone = a @ a
+    torch.cuda.synchronize()
+    assert torch.allclose(c.float(), c_alone.float(), rtol=1e-2, atol=1e-2)
     lay = oracle.layout(topk, wl.E, wl.pad, buf.cap)
     used = int(lay["offsets"][-1])
     np.testing.assert_array_equal(hd.pos.cpu().numpy(), lay["pos"])
