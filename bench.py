@@ -386,6 +386,17 @@ class Path:
         self.ep.ep_combine(self.y, self.pos, io["w"], wl.N, wl.K, wl.H,
                            io["out"], status=self.status, cap=self.cap)
 
+    def combine_recv_weights(self, io=None):
+        """The combine with receive-side weights (the EPBuffer call)."""
+        wl = self.wl
+        io = io or self.io()
+        if not hasattr(self, "gathered"):
+            self.gathered = torch.empty(wl.N, wl.K, dtype=torch.float32,
+                                        device=self.dev)
+        self.ep.ep_combine_recv_weights(self.y, self.pos, self.recv_w, wl.N,
+                                        wl.K, wl.H, io["out"], self.gathered,
+                                        status=self.status, cap=self.cap)
+
     def step(self, io=None):
         self.layout_dispatch(io)
         if self.wl.B > 0:
@@ -509,7 +520,7 @@ def measure(paths, K, warmup, backward, device_index, flush, barrier=None,
 
     calls = ["layout_dispatch", "combine"]
     if kernels:
-        calls += ["layout", "dispatch"]
+        calls += ["layout", "dispatch", "combine_recv_weights"]
     if wl.B:
         calls.append("plan_prefetch")
     if backward:
@@ -813,6 +824,8 @@ def run_gpu(args, wl):
                 "layout_us": round(avg["layout"], 2),
                 "dispatch_us": round(avg["dispatch"], 2),
                 "combine_us": round(avg["combine"], 2),
+                "combine_recv_weights_us": round(
+                    avg.get("combine_recv_weights", 0.0), 2),
                 "plan_prefetch_us": round(avg.get("plan_prefetch", 0.0), 2),
                 "layout_plus_dispatch_us": round(avg["layout"] +
                                                  avg["dispatch"], 2),

@@ -209,15 +209,21 @@ __global__ void __launch_bounds__((kTmaMaxConsumerWarps + 1) * 32, 1)
 
   if (warp == cw) {
     // ---- producer warp: lane k handles the k-th gathered part-row --------
+    // Positions run two units ahead and weights one: a receive-side weight
+    // is read at its entry's row, so its load waits for the position, which
+    // was loaded an iteration earlier. Both loads go out before the wait
+    // for a free stage, which hides their latency.
     int it = 0;
     int64_t u = blockIdx.x;
-    int p_n = -1;
+    int p_n = -1, p_nn = -1;
     float w_n = 0.0f;
     if (u < units && lane < K) {
       const int64_t t0 = u / sh.parts;
       p_n = __ldg(pos + t0 * K + lane);
       w_n = entry_weight(wts, t0, K, lane, p_n, cap);
     }
+    if (u + gridDim.x < units && lane < K)
+      p_nn = __ldg(pos + ((u + gridDim.x) / sh.parts) * K + lane);
     for (; u < units; u += gridDim.x, ++it) {
       const int64_t t = u / sh.parts;
       const int part = int(u - t * sh.parts);
@@ -226,13 +232,13 @@ __global__ void __launch_bounds__((kTmaMaxConsumerWarps + 1) * 32, 1)
       const uint32_t bytes = uint32_t(len) * 2u;
       const int p = p_n;
       const float wv = w_n;
-      {  // positions of the next unit, one unit ahead
-        const int64_t un = u + gridDim.x;
+      {  // the next unit's weight, and the position of the one after
+        const int64_t un = u + gridDim.x, unn = un + gridDim.x;
         if (un < units && lane < K) {
-          const int64_t tn = un / sh.parts;
-          p_n = __ldg(pos + tn * K + lane);
-          w_n = entry_weight(wts, tn, K, lane, p_n, cap);
+          p_n = p_nn;
+          w_n = entry_weight(wts, un / sh.parts, K, lane, p_n, cap);
         }
+        if (unn < units && lane < K) p_nn = __ldg(pos + (unn / sh.parts) * K + lane);
       }
       if (wts.rows && wts.gathered && part == 0 && lane < K)
         wts.gathered[t * K + lane] = wv;
