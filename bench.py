@@ -727,24 +727,30 @@ def run_gpu(args, wl):
         with nvtx(f"{wl.name}: end to end"):
             e2e = run_e2e(args, path, b["step"], rank_max, barrier)
 
-    # a streaming read of 4 GiB (torch's reduction kernel), timed here as
-    # context for read-heavy calls, whose rate can exceed the copy peak
-    read_probe = None
+    # a streaming read and a streaming write of 4 GiB (torch's reduction
+    # and fill kernels), timed here as context: a read-heavy call such as
+    # combine can pass the copy peak, a write-heavy one such as dispatch is
+    # bounded by the write rate
+    read_probe = write_probe = None
     if rank == 0 and not args.no_read_probe:
-        with nvtx("read probe"):
+        with nvtx("read / write probes"):
             x = torch.empty(4 << 30, dtype=torch.uint8, device=dev).view(
                 torch.int64)
-            x.fill_(1)
-            for _ in range(2):
-                x.max()
-            a_, b_ = (torch.cuda.Event(enable_timing=True),
-                      torch.cuda.Event(enable_timing=True))
-            a_.record()
-            for _ in range(5):
-                x.max()
-            b_.record()
-            torch.cuda.synchronize()
-            read_probe = (4 << 30) * 5 / (a_.elapsed_time(b_) * 1e-3) / 1e9
+
+            def rate(fn):
+                for _ in range(2):
+                    fn()
+                a_, b_ = (torch.cuda.Event(enable_timing=True),
+                          torch.cuda.Event(enable_timing=True))
+                a_.record()
+                for _ in range(5):
+                    fn()
+                b_.record()
+                torch.cuda.synchronize()
+                return (4 << 30) * 5 / (a_.elapsed_time(b_) * 1e-3) / 1e9
+
+            write_probe = rate(lambda: x.fill_(1))
+            read_probe = rate(lambda: x.max())
             del x
 
     epbuf = None
@@ -878,10 +884,16 @@ def run_gpu(args, wl):
                                     else None),
                 "frac_of_read_probe": (round(dom_gbs / read_probe, 4)
                                        if read_probe else None),
+                "write_probe_GBps": (round(write_probe, 1) if write_probe
+                                     else None),
+                "dispatch_frac_of_write_probe": (
+                    round(dis_gbs / write_probe, 4) if write_probe else None),
                 "note": "peak is a copy (half reads, half writes); a "
                         "read-heavy call such as combine (89% reads) can "
                         "pass it, so the same call is also given against a "
-                        "4 GiB streaming read timed in this run",
+                        "4 GiB streaming read timed in this run, and the "
+                        "write-heavy dispatch (80% writes) against a 4 GiB "
+                        "streaming write",
             },
             "clocks": clocks,
             "e2e": e2e,
@@ -1129,7 +1141,7 @@ def main():
     ap.add_argument("--no-extra-workloads", action="store_true",
                     help="time only the selected workload")
     ap.add_argument("--no-read-probe", action="store_true",
-                    help="skip the 4 GiB streaming-read probe")
+                    help="skip the 4 GiB streaming read and write probes")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--backward", action="store_true",
                     help="add the backward pair to the step")
