@@ -923,6 +923,20 @@ def run_gpu(args, wl):
             del xp
             torch.cuda.empty_cache()
     if result is not None and extras:
+        # the decode step's receive rows stay in L2: its layout + dispatch
+        # call is given against an L2-resident write as well (a graph of
+        # 20 fills of one 64 MB buffer)
+        if "decode" in extras and not args.no_read_probe:
+            x = torch.empty(64 << 20, dtype=torch.uint8, device=dev)
+            x.fill_(1)
+            g = capture(lambda i: x.fill_(i & 1), 20)
+            replay_ms(g)
+            l2w = (64 << 20) * 20 / (replay_ms(g) * 1e-3) / 1e9
+            del g, x
+            dec = extras["decode"]
+            ld = dec["rates"]["layout_dispatch"]
+            dec["l2_write_probe_GBps"] = round(l2w, 1)
+            ld["frac_of_l2_write_probe"] = round(ld["GBps"] / l2w, 4)
         result["workloads"] = extras
     del flush
     if ws > 1:
