@@ -83,3 +83,18 @@ def test_combine_kernel_follows_the_library_rule(N, K, H, expect):
     wl = workloads.scaled(workloads.WORKLOADS["prefill"], S=N // 8, K=K, H=H)
     wl = workloads.scaled(wl, R=1, S=N)
     assert bench.combine_kernel(wl) == expect
+
+
+def test_dispatch_kernel_names_follow_the_library_rule():
+    src = open(os.path.join(ROOT, "combine_ep_layout_09_b200", "csrc",
+                            "dispatch.cu")).read()
+    # with every SM in use a bf16 dispatch launches one CTA per token
+    assert re.search(r"all_sms\s*=\s*num_sms\s*>=\s*device_sm_count\(\)", src)
+    assert re.search(r"if\s*\(all_sms\s*&&\s*!fp8\)", src)
+    for name in ("k_dispatch_bf16_tok", "k_dispatch_fp8"):
+        assert re.search(r"cudaLaunchKernelEx\(&cfg,\s*" + name + ",", src)
+    names = {w: bench.kernel_names(workloads.WORKLOADS[w])["dispatch"]
+             for w in ("prefill", "skewed", "decode")}
+    assert names == {"prefill": "k_dispatch_fp8",
+                     "skewed": "k_dispatch_bf16_tok",
+                     "decode": "k_layout_small<fp8>"}

@@ -153,9 +153,12 @@ def test_dispatch_waits_give_up(fp8):
     def run():
         recv, scales, recv_w = dispatch_bufs(cap, H, fp8)
         st = status_tensor()
+        # on fewer SMs than the device has the dispatch runs its persistent
+        # kernels, the ones with waits (on every SM it runs one CTA per
+        # token, which waits on nothing)
         ep.ep_dispatch(hid, wd, g["dev"]["pos"], g["dev"]["row_src"],
                        g["dev"]["offsets"], N, K, E, H, fp8, recv, scales,
-                       recv_w, status=st, cap=cap)
+                       recv_w, num_sms=100, status=st, cap=cap)
         torch.cuda.synchronize()
         return recv, scales, recv_w, int(st[0].item())
 
@@ -168,8 +171,9 @@ def test_dispatch_waits_give_up(fp8):
     check_dispatch(recv, scales, recv_w, topk, w, h, E, pad, cap, fp8)
 
 
-@pytest.mark.parametrize("fp8", [False, True])
-def test_layout_dispatch_large_batch_gives_up(fp8):
+@pytest.mark.parametrize("fp8,num_sms", [(False, 0), (True, 0), (False, 100),
+                                         (True, 100)])
+def test_layout_dispatch_large_batch_gives_up(fp8, num_sms):
     # the layout kernel, then the dispatch kernel launched as its programmatic
     # dependent; both sites forced at once
     E, pad, H, R = 64, 1, 1024, 4
@@ -185,7 +189,7 @@ def test_layout_dispatch_large_batch_gives_up(fp8):
         ep.ep_layout_dispatch(t, hid, wd, R, S, K, E, H, pad, fp8, b["counts"],
                               b["offsets"], b["pos"], b["row_src"], recv,
                               scales, recv_w, workspace=b["ws"],
-                              status=b["status"], cap=cap)
+                              num_sms=num_sms, status=b["status"], cap=cap)
         torch.cuda.synchronize()
         return b, recv, scales, recv_w
 
