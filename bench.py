@@ -590,11 +590,9 @@ def kernel_names(wl, sms=148):
     prec = "fp8" if wl.fp8 else "bf16"
     if one_launch:
         disp = f"k_layout_small<{prec}>"
-    elif wl.fp8:
-        disp = "k_dispatch_fp8"
     else:
         # a grid of one CTA per token when every SM is in use
-        disp = "k_dispatch_bf16_tok"
+        disp = f"k_dispatch_{prec}_tok"
     return {"one_launch": one_launch, "dispatch": disp,
             "combine": combine_kernel(wl, sms)}
 

@@ -8,10 +8,21 @@
 // directly in their final expert-grouped position (computed by the layout
 // kernels), with no later permutation.
 //
-// Both kernels move rows with the TMA engine's 1-D bulk copies (no tensor
-// map; each CTA loads only its own rows): a token row comes into shared
-// memory once and leaves K times. The kernel reads 1/(K+1) of the bytes it
-// moves, so HBM write bandwidth bounds it.
+// A token row is read once and written K times, so the kernels read
+// 1/(K+1) of the bytes they move (bf16) and HBM write bandwidth bounds them.
+// With every SM in use, one CTA per token:
+//
+//   k_dispatch_bf16_tok  each thread loads 16-byte vectors of the row and
+//                        stores each to the K rows.
+//   k_dispatch_fp8_tok   each warp loads two 512-channel units, quantises
+//                        them in registers and stores codes and scales to
+//                        the K rows.
+//
+// Short CTAs start in token order, so the rows being written at any moment
+// belong to a narrow window of tokens. A grid of short CTAs cannot be held
+// to fewer SMs, so a num_sms limit takes the persistent kernels, which move
+// rows with the TMA engine's 1-D bulk copies (no tensor map; each CTA loads
+// only its own rows):
 //
 //   k_dispatch_bf16  one-warp CTAs; lane 0 keeps a ring of token rows in
 //                    flight and, per row, issues K bulk stores from shared
@@ -358,6 +369,89 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32)
   zero_padding_rows<false>(row_src, offsets, E, H, cap, recv, nullptr, recv_w);
 }
 
+// ---------------------------------------------------------------------------
+// FP8, one token per CTA (every SM in use): each warp loads two 512-channel
+// units of the row with 16-byte loads before it quantises either, then
+// quantises each unit in registers (a lane's 16 channels, 8 lanes per
+// 128-channel group, as in the persistent kernel) and stores its 16 codes to
+// the K rows; lanes 8g store the group's scale. 224 threads cover H=7168, so
+// four CTAs share an SM: four token rows in flight per SM, written in token
+// order as in the bf16 form.
+// ---------------------------------------------------------------------------
+
+constexpr int kFp8TokUnits = 2;     // 512-channel units a warp holds at once
+constexpr int kFp8TokMaxWarps = 7;  // H/1024 rounded up, capped (H=7168)
+
+__global__ void __launch_bounds__(kFp8TokMaxWarps * 32, 4)
+    k_dispatch_fp8_tok(const uint16_t* __restrict__ hidden,
+                       const float* __restrict__ w,
+                       const int32_t* __restrict__ pos,
+                       const int32_t* __restrict__ row_src,
+                       const int32_t* __restrict__ offsets, int64_t N, int K,
+                       int E, int H, int64_t cap, uint8_t* __restrict__ recv,
+                       float* __restrict__ scales, float* __restrict__ recv_w,
+                       int32_t* __restrict__ status) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
+  const int G = H >> 7;
+  bool waited = false;
+  for (int64_t t = blockIdx.x; t < N; t += gridDim.x) {
+    const uint16_t* row = hidden + t * H;
+    // warp-uniform loop over passes of nwarps * kFp8TokUnits units
+    for (int u0 = warp; u0 * kUnitCh < H; u0 += nwarps * kFp8TokUnits) {
+      uint4 a[kFp8TokUnits], b[kFp8TokUnits];
+#pragma unroll
+      for (int j = 0; j < kFp8TokUnits; ++j) {
+        const int c0 = (u0 + j * nwarps) * kUnitCh + lane * 16;
+        a[j] = b[j] = make_uint4(0u, 0u, 0u, 0u);
+        if (c0 < H) {
+          a[j] = ld_stream_v4(row + c0);
+          b[j] = ld_stream_v4(row + c0 + 8);
+        }
+      }
+      // the rows do not depend on the layout ahead; the positions do
+      if (!waited) {
+        grid_dependency_wait();
+        waited = true;
+      }
+      int p_l = -1;
+      if (lane < K) {
+        p_l = __ldg(pos + t * K + lane);
+        if (p_l >= cap) {
+          if (warp == 0 && u0 == warp) report(status, EP_DEV_CAPACITY);
+          p_l = -1;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kFp8TokUnits; ++j) {
+        const int c0 = (u0 + j * nwarps) * kUnitCh + lane * 16;
+        const bool act = c0 < H;  // H % 128 == 0: whole groups
+        float x[16];
+        float amax = unpack16(a[j], b[j], x);
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+        const float scale = __fdiv_rn(amax, 448.0f);
+        uint4 q = make_uint4(0u, 0u, 0u, 0u);
+        if (scale != 0.0f) q = quantize16(x, make_group_scale(scale));
+        for (int k = 0; k < K; ++k) {
+          const int p = __shfl_sync(0xffffffffu, p_l, k);
+          if (act && p >= 0) {
+            st_v4(recv + int64_t(p) * H + c0, q);
+            if ((lane & 7) == 0) scales[int64_t(p) * G + (c0 >> 7)] = scale;
+          }
+        }
+      }
+    }
+    if (warp == 0 && lane < K && recv_w) {
+      const int p = __ldg(pos + t * K + lane);
+      if (p >= 0 && p < cap) recv_w[p] = __ldg(w + t * K + lane);
+    }
+  }
+  if (!waited) grid_dependency_wait();  // row_src / offsets from the layout
+  zero_padding_rows<true>(row_src, offsets, E, H, cap, recv, scales, recv_w);
+}
+
 __global__ void k_debug_quantize(const float* __restrict__ x,
                                  const float* __restrict__ scale,
                                  uint8_t* __restrict__ out, int64_t n) {
@@ -424,6 +518,24 @@ cudaError_t launch_dispatch(const void* hidden, const float* w,
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   const bool all_sms = num_sms >= device_sm_count();
+  if (all_sms && fp8) {
+    // FP8 on every SM: one CTA per token, as for bf16 below
+    const int units = (H + kUnitCh - 1) / kUnitCh;
+    const int warps = std::min(
+        kFp8TokMaxWarps, (units + kFp8TokUnits - 1) / kFp8TokUnits);
+    const int64_t pad_ctas = ((cap + 31) / 32 + warps - 1) / warps;
+    const int64_t grid = std::max<int64_t>(
+        1, std::min<int64_t>(INT32_MAX, std::max<int64_t>(N, pad_ctas)));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(grid));
+    cfg.blockDim = dim3(unsigned(warps * 32));
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, k_dispatch_fp8_tok, h, w, pos, row_src,
+                              expert_offsets, N, K, E, H, cap, r, recv_scales,
+                              recv_w, status);
+  }
   if (all_sms && !fp8) {
     // bf16 on every SM: one CTA per token (a grid of N short CTAs cannot be
     // held to fewer SMs, so a num_sms limit takes the persistent kernel)
@@ -455,9 +567,7 @@ cudaError_t launch_dispatch(const void* hidden, const float* w,
   if (err != cudaSuccess) return err;
   per_sm = std::max(1, per_sm);
   // Persistent CTAs on the SMs allowed, each taking every grid-th token:
-  // enough CTAs for the token rows and for the padding sweep. (Short CTAs of
-  // 4-32 consecutive tokens were measured slower for FP8: 448-523 us
-  // against 426 us on the prefill batch.)
+  // enough CTAs for the token rows and for the padding sweep.
   const int64_t grid = std::max<int64_t>(
       1, std::min<int64_t>(int64_t(num_sms) * per_sm,
                            std::max<int64_t>(N, (cap + 31) / 32)));

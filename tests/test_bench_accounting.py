@@ -88,13 +88,14 @@ def test_combine_kernel_follows_the_library_rule(N, K, H, expect):
 def test_dispatch_kernel_names_follow_the_library_rule():
     src = open(os.path.join(ROOT, "combine_ep_layout_09_b200", "csrc",
                             "dispatch.cu")).read()
-    # with every SM in use a bf16 dispatch launches one CTA per token
+    # with every SM in use the dispatch launches one CTA per token
     assert re.search(r"all_sms\s*=\s*num_sms\s*>=\s*device_sm_count\(\)", src)
     assert re.search(r"if\s*\(all_sms\s*&&\s*!fp8\)", src)
-    for name in ("k_dispatch_bf16_tok", "k_dispatch_fp8"):
+    assert re.search(r"if\s*\(all_sms\s*&&\s*fp8\)", src)
+    for name in ("k_dispatch_bf16_tok", "k_dispatch_fp8_tok"):
         assert re.search(r"cudaLaunchKernelEx\(&cfg,\s*" + name + ",", src)
     names = {w: bench.kernel_names(workloads.WORKLOADS[w])["dispatch"]
              for w in ("prefill", "skewed", "decode")}
-    assert names == {"prefill": "k_dispatch_fp8",
+    assert names == {"prefill": "k_dispatch_fp8_tok",
                      "skewed": "k_dispatch_bf16_tok",
                      "decode": "k_layout_small<fp8>"}

@@ -45,6 +45,9 @@ def check_full(topk, w, hidden, R, S, E, H, pad, fp8, num_sms=0,
         np.testing.assert_array_equal(d["recv_w"].cpu().numpy()[:cap], rw)
 
 
+# num_sms 0: one CTA per token; 100 (fewer SMs than the device has): the
+# persistent kernels
+@pytest.mark.parametrize("num_sms", [0, 100])
 @pytest.mark.parametrize("R,S,K,E,H,pad", [
     (4, 64, 2, 8, 256, 1),          # tiny shape
     (2, 700, 8, 16, 7168, 1),       # several tiles, full row width
@@ -53,11 +56,12 @@ def check_full(topk, w, hidden, R, S, E, H, pad, fp8, num_sms=0,
     (4, 100, 4, 16, 24, 128),       # odd vector count, heavy padding
     (1, 1, 1, 1, 16, 1),
 ])
-def test_bf16(R, S, K, E, H, pad):
+def test_bf16(R, S, K, E, H, pad, num_sms):
     topk, w, h = make(R + S + K + E + H, R, S, K, E, H)
-    check_full(topk, w, h, R, S, E, H, pad, fp8=False)
+    check_full(topk, w, h, R, S, E, H, pad, fp8=False, num_sms=num_sms)
 
 
+@pytest.mark.parametrize("num_sms", [0, 100])
 @pytest.mark.parametrize("R,S,K,E,H,pad", [
     (4, 64, 2, 8, 256, 1),
     (2, 700, 8, 16, 7168, 1),
@@ -65,12 +69,13 @@ def test_bf16(R, S, K, E, H, pad):
     (2, 301, 8, 32, 640, 128),
     (1, 1, 1, 1, 128, 1),
 ])
-def test_fp8(R, S, K, E, H, pad):
+def test_fp8(R, S, K, E, H, pad, num_sms):
     topk, w, h = make(7 * (R + S + K + E + H), R, S, K, E, H)
-    check_full(topk, w, h, R, S, E, H, pad, fp8=True)
+    check_full(topk, w, h, R, S, E, H, pad, fp8=True, num_sms=num_sms)
 
 
-def test_fp8_extreme_values():
+@pytest.mark.parametrize("num_sms", [0, 100])
+def test_fp8_extreme_values(num_sms):
     # huge, tiny, subnormal and zero groups, signed zeros, exact ties
     R, S, K, E, H = 2, 40, 3, 4, 512
     rng = np.random.default_rng(3)
@@ -86,7 +91,7 @@ def test_fp8_extreme_values():
     x[5, :] = 3e-39                        # bf16 subnormal group
     x[6, ::2] = -x[6, ::2]
     h = (x.view(np.uint32) >> 16).astype(np.uint16)   # truncate to bf16
-    check_full(topk, w, h, R, S, E, H, 1, fp8=True)
+    check_full(topk, w, h, R, S, E, H, 1, fp8=True, num_sms=num_sms)
 
 
 @pytest.mark.parametrize("fp8", [False, True])
@@ -109,11 +114,13 @@ def test_k32(fp8):
     check_full(topk, w, h, 2, 200, 64, 256, 1, fp8=fp8)
 
 
+@pytest.mark.parametrize("num_sms", [0, 100])
 @pytest.mark.parametrize("fp8", [False, True])
-def test_widest_row(fp8):
-    # H = 32768, the largest the ABI accepts: two input stages of 64 KB
+def test_widest_row(fp8, num_sms):
+    # H = 32768, the largest the ABI accepts: two input stages of 64 KB in
+    # the persistent kernels, several passes of a CTA's warps per token
     topk, w, h = make(322, 1, 48, 3, 4, 32768)
-    check_full(topk, w, h, 1, 48, 4, 32768, 1, fp8=fp8)
+    check_full(topk, w, h, 1, 48, 4, 32768, 1, fp8=fp8, num_sms=num_sms)
 
 
 @pytest.mark.parametrize("fp8", [False, True])
