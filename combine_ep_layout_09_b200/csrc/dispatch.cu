@@ -329,6 +329,7 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 2)
 // CTA per token against 5.9-6.1 TB/s from persistent CTAs).
 // ---------------------------------------------------------------------------
 
+template <bool kWide>
 __global__ void __launch_bounds__(kMaxConsumerWarps * 32)
     k_dispatch_bf16_tok(const uint16_t* __restrict__ hidden,
                         const float* __restrict__ w,
@@ -339,7 +340,8 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32)
                         float* __restrict__ recv_w,
                         int32_t* __restrict__ status) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int V = H >> 3;  // 16-byte vectors of a row
+  constexpr int kVec = kWide ? 16 : 8;  // channels a thread moves at once
+  const int V = H / kVec;               // vectors of a row
   uint16_t* recv16 = reinterpret_cast<uint16_t*>(recv);
   grid_dependency_wait();  // pos / row_src / offsets may come from the layout
   for (int64_t t = blockIdx.x; t < N; t += gridDim.x) {
@@ -357,11 +359,21 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32)
     // warp-uniform loop: every lane takes part in the shuffles
     for (int v0 = warp * 32; v0 < V; v0 += blockDim.x) {
       const int v = v0 + lane;
-      uint4 d = make_uint4(0u, 0u, 0u, 0u);
-      if (v < V) d = ld_stream_v4(row + v * 8);
+      uint4 d = make_uint4(0u, 0u, 0u, 0u), d1 = d;
+      if (v < V) {
+        if constexpr (kWide)
+          ld_stream_v8(row + v * kVec, d, d1);
+        else
+          d = ld_stream_v4(row + v * kVec);
+      }
       for (int k = 0; k < K; ++k) {
         const int p = __shfl_sync(0xffffffffu, p_l, k);
-        if (p >= 0 && v < V) st_v4(recv16 + int64_t(p) * H + v * 8, d);
+        if (p >= 0 && v < V) {
+          if constexpr (kWide)
+            st_v8(recv16 + int64_t(p) * H + v * kVec, d, d1);
+          else
+            st_v4(recv16 + int64_t(p) * H + v * kVec, d);
+        }
       }
     }
     if (warp == 0 && lane < K && p_l >= 0 && recv_w) recv_w[p_l] = w_l;
@@ -382,6 +394,7 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32)
 constexpr int kFp8TokUnits = 2;     // 512-channel units a warp holds at once
 constexpr int kFp8TokMaxWarps = 7;  // H/1024 rounded up, capped (H=7168)
 
+template <bool kWide>
 __global__ void __launch_bounds__(kFp8TokMaxWarps * 32, 4)
     k_dispatch_fp8_tok(const uint16_t* __restrict__ hidden,
                        const float* __restrict__ w,
@@ -405,8 +418,12 @@ __global__ void __launch_bounds__(kFp8TokMaxWarps * 32, 4)
         const int c0 = (u0 + j * nwarps) * kUnitCh + lane * 16;
         a[j] = b[j] = make_uint4(0u, 0u, 0u, 0u);
         if (c0 < H) {
-          a[j] = ld_stream_v4(row + c0);
-          b[j] = ld_stream_v4(row + c0 + 8);
+          if constexpr (kWide) {
+            ld_stream_v8(row + c0, a[j], b[j]);
+          } else {
+            a[j] = ld_stream_v4(row + c0);
+            b[j] = ld_stream_v4(row + c0 + 8);
+          }
         }
       }
       // the rows do not depend on the layout ahead; the positions do
@@ -431,7 +448,7 @@ __global__ void __launch_bounds__(kFp8TokMaxWarps * 32, 4)
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
         amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-        const float scale = __fdiv_rn(amax, 448.0f);
+        const float scale = scale_of_amax(amax);
         uint4 q = make_uint4(0u, 0u, 0u, 0u);
         if (scale != 0.0f) q = quantize16(x, make_group_scale(scale));
         for (int k = 0; k < K; ++k) {
@@ -518,6 +535,9 @@ cudaError_t launch_dispatch(const void* hidden, const float* w,
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   const bool all_sms = num_sms >= device_sm_count();
+  // 32-byte accesses where every row start is 32-byte aligned
+  const bool in32 = (reinterpret_cast<uintptr_t>(hidden) & 31u) == 0;
+  const bool out32 = (reinterpret_cast<uintptr_t>(recv) & 31u) == 0;
   if (all_sms && fp8) {
     // FP8 on every SM: one CTA per token, as for bf16 below
     const int units = (H + kUnitCh - 1) / kUnitCh;
@@ -532,14 +552,16 @@ cudaError_t launch_dispatch(const void* hidden, const float* w,
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, k_dispatch_fp8_tok, h, w, pos, row_src,
-                              expert_offsets, N, K, E, H, cap, r, recv_scales,
-                              recv_w, status);
+    // H % 128 == 0: every row start is as aligned as the buffer
+    auto kern = in32 ? k_dispatch_fp8_tok<true> : k_dispatch_fp8_tok<false>;
+    return cudaLaunchKernelEx(&cfg, kern, h, w, pos, row_src, expert_offsets,
+                              N, K, E, H, cap, r, recv_scales, recv_w, status);
   }
   if (all_sms && !fp8) {
     // bf16 on every SM: one CTA per token (a grid of N short CTAs cannot be
     // held to fewer SMs, so a num_sms limit takes the persistent kernel)
-    const int V = H >> 3;
+    const bool wide = in32 && out32 && H % 16 == 0;
+    const int V = wide ? H >> 4 : H >> 3;
     const int passes = (V + kMaxConsumerWarps * 32 - 1) / (kMaxConsumerWarps * 32);
     const int threads = std::max(32, ((V + passes - 1) / passes + 31) / 32 * 32);
     const int64_t pad_ctas = ((cap + 31) / 32 + threads / 32 - 1) / (threads / 32);
@@ -551,9 +573,9 @@ cudaError_t launch_dispatch(const void* hidden, const float* w,
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, k_dispatch_bf16_tok, h, w, pos, row_src,
-                              expert_offsets, N, K, E, H, cap, r, recv_w,
-                              status);
+    auto kern = wide ? k_dispatch_bf16_tok<true> : k_dispatch_bf16_tok<false>;
+    return cudaLaunchKernelEx(&cfg, kern, h, w, pos, row_src, expert_offsets,
+                              N, K, E, H, cap, r, recv_w, status);
   }
   const Cfg c = fp8 ? fp8_cfg(H) : bf16_cfg(H);
   const void* kern = fp8 ? reinterpret_cast<const void*>(k_dispatch_fp8)

@@ -106,6 +106,23 @@ __device__ __forceinline__ void st_v4(void* p, uint4 v) {
                : "memory");
 }
 
+// 32-byte forms (256-bit global accesses, sm_100): p must be 32-byte aligned.
+__device__ __forceinline__ void ld_stream_v8(const void* p, uint4& lo,
+                                             uint4& hi) {
+  asm volatile(
+      "ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+      : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x),
+        "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+      : "l"(p));
+}
+
+__device__ __forceinline__ void st_v8(void* p, uint4 lo, uint4 hi) {
+  asm volatile("st.global.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p),
+               "r"(lo.x), "r"(lo.y), "r"(lo.z), "r"(lo.w), "r"(hi.x),
+               "r"(hi.y), "r"(hi.z), "r"(hi.w)
+               : "memory");
+}
+
 // Streaming store (evict-first): the receive buffer is far larger than L2.
 __device__ __forceinline__ void st_cs_v4(void* p, uint4 v) {
   asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x),

@@ -93,7 +93,8 @@ def test_dispatch_kernel_names_follow_the_library_rule():
     assert re.search(r"if\s*\(all_sms\s*&&\s*!fp8\)", src)
     assert re.search(r"if\s*\(all_sms\s*&&\s*fp8\)", src)
     for name in ("k_dispatch_bf16_tok", "k_dispatch_fp8_tok"):
-        assert re.search(r"cudaLaunchKernelEx\(&cfg,\s*" + name + ",", src)
+        assert re.search(r"auto kern = \w+ \? " + name + r"<true> : " + name +
+                         r"<false>;", src)
     names = {w: bench.kernel_names(workloads.WORKLOADS[w])["dispatch"]
              for w in ("prefill", "skewed", "decode")}
     assert names == {"prefill": "k_dispatch_fp8_tok",

@@ -94,6 +94,28 @@ def test_fp8_extreme_values(num_sms):
     check_full(topk, w, h, R, S, E, H, 1, fp8=True, num_sms=num_sms)
 
 
+@pytest.mark.parametrize("num_sms", [0, 100])
+def test_fp8_scale_for_every_bf16_amax(num_sms):
+    # one 128-channel group per finite non-negative bf16 value v: its largest
+    # magnitude is v (signs alternate), so the kernels' scale RN(v/448) is
+    # checked against the oracle's division for every amax a bf16 row can
+    # have, and the group's codes with it
+    H, G = 7168, 56
+    vals = (np.arange(0, 0x7f80, dtype=np.uint32) << 16).view(np.float32)
+    n_groups = -(-len(vals) // G) * G
+    amax = np.resize(vals, n_groups)
+    rng = np.random.default_rng(11)
+    x = amax[:, None] * rng.uniform(-1.0, 1.0, (n_groups, 128)).astype(np.float32)
+    x[:, 0] = amax * np.where(np.arange(n_groups) % 2 == 0, 1.0, -1.0)
+    # truncate to bf16: magnitudes never rise above the group's amax
+    h = (np.ascontiguousarray(x, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    h = h.reshape(-1, H)
+    N = h.shape[0]
+    topk = np.zeros((N, 1), np.int32)
+    w = rng.random((N, 1)).astype(np.float32)
+    check_full(topk, w, h, 1, N, 1, H, 1, fp8=True, num_sms=num_sms)
+
+
 @pytest.mark.parametrize("fp8", [False, True])
 def test_without_weights_and_limited_sms(fp8):
     topk, w, h = make(99, 2, 500, 4, 8, 1024)
