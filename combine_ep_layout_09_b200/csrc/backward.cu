@@ -12,7 +12,8 @@
 // dispatch backward:  grad_hidden[t] = bf16( sum_k grad_recv[pos[t,k]] )
 //                     (combine with unit weights: launch_combine, w = NULL)
 //
-// k_combine_bwd: persistent CTAs walk tokens; threads split the row into
+// k_combine_bwd: CTAs walk tokens (one CTA per token when every SM is in
+// use, persistent CTAs under a num_sms limit); threads split the row into
 // 16-byte vectors. Each thread loads the grad_out vector and its K gathered
 // expert-output vectors, accumulates the K dot products in fp32 (its
 // vectors in order, channels in order), and stores the K scaled gradient
@@ -158,9 +159,15 @@ cudaError_t launch_combine_backward(const void* grad_out, const void* y,
   cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
       &per_sm, k_combine_bwd, threads, 0);
   if (err != cudaSuccess) return err;
+  // Every SM in use: one CTA per token, so that the CTAs start in token
+  // order and the rows written at any moment belong to a narrow window of
+  // tokens. A num_sms limit keeps persistent CTAs (a grid of short CTAs
+  // cannot be held to fewer SMs).
+  const int64_t resident = num_sms >= device_sm_count()
+                               ? int64_t(INT32_MAX)
+                               : int64_t(num_sms) * std::max(1, per_sm);
   const int64_t grid = std::max<int64_t>(
-      1, std::min<int64_t>(int64_t(num_sms) * std::max(1, per_sm),
-                           std::max<int64_t>(N, (cap + 31) / 32)));
+      1, std::min<int64_t>(resident, std::max<int64_t>(N, (cap + 31) / 32)));
   k_combine_bwd<<<int(grid), threads, 0, stream>>>(
       static_cast<const uint16_t*>(grad_out), static_cast<const uint16_t*>(y),
       pos, row_src, expert_offsets, w, N, K, E, H, cap,

@@ -39,7 +39,7 @@ def test_dispatch_backward(N, K, H, rows):
     np.testing.assert_array_equal(u16(out), oracle.dispatch_backward(g, pos))
 
 
-def run_combine_backward(topk, w, R, S, E, H, pad, seed):
+def run_combine_backward(topk, w, R, S, E, H, pad, seed, num_sms=0):
     N, K = topk.shape
     lay = gpu_layout(topk, R, S, E, pad)
     cap = lay["dev"]["cap"]
@@ -51,7 +51,7 @@ def run_combine_backward(topk, w, R, S, E, H, pad, seed):
     st = status_tensor()
     ep.ep_combine_backward(g, y, lay["dev"]["pos"], lay["dev"]["row_src"],
                            lay["dev"]["offsets"], to_dev(w), N, K, E, H, rows,
-                           gw, status=st)
+                           gw, num_sms=num_sms, status=st)
     torch.cuda.synchronize()
     assert int(st[0].item()) == 0
     return lay, cap, y, g, rows, gw
@@ -66,15 +66,17 @@ def weight_grad_ok(got, g_bits, y_rows_bits, K, H):
     assert np.all(np.abs(got - exact) <= H * 2.0 ** -24 * mag + 1e-30)
 
 
+# num_sms 0: one CTA per token; 100: persistent CTAs on fewer SMs
+@pytest.mark.parametrize("num_sms", [0, 100])
 @pytest.mark.parametrize("R,S,K,E,H,pad", [
     (4, 64, 2, 8, 256, 1), (2, 300, 8, 16, 7168, 4), (3, 200, 5, 9, 520, 128),
 ])
-def test_combine_backward_small(R, S, K, E, H, pad):
+def test_combine_backward_small(R, S, K, E, H, pad, num_sms):
     rng = np.random.default_rng(R * S + K)
     topk, w = workloads.random_topk(rng, R * S, K, E)
     w = (w * rng.choice([-1.0, 1.0], w.shape) * 2).astype(np.float32)
     lay, cap, y, g, rows, gw = run_combine_backward(topk, w, R, S, E, H, pad,
-                                                     R + S)
+                                                     R + S, num_sms=num_sms)
     o = oracle.layout(topk, E, pad, cap)
     ref_rows = oracle.combine_backward_rows(u16(g), w, o, E, cap,
                                             fill=RECV_BF16_FILL)
