@@ -7,8 +7,11 @@ import torch
 
 import oracle
 import workloads
-from gpu_util import (RECV_BF16_FILL, RECV_FP8_FILL, RECV_W_FILL, SCALE_FILL,
-                      gpu_dispatch, gpu_layout, to_bf16_dev, u16)
+from gpu_util import (DEV, RECV_BF16_FILL, RECV_FP8_FILL, RECV_W_FILL,
+                      SCALE_FILL, gpu_dispatch, gpu_layout, status_tensor,
+                      to_bf16_dev, to_dev, u16)
+
+import combine_ep_layout_09_b200 as ep
 
 pytestmark = pytest.mark.gpu
 
@@ -114,6 +117,55 @@ def test_fp8_scale_for_every_bf16_amax(num_sms):
     topk = np.zeros((N, 1), np.int32)
     w = rng.random((N, 1)).astype(np.float32)
     check_full(topk, w, h, 1, N, 1, H, 1, fp8=True, num_sms=num_sms)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_rows_16_byte_aligned_only(fp8):
+    # hidden and the receive rows start 16 bytes past a 32-byte boundary, so
+    # the per-token kernels take their 16-byte access forms
+    R, S, K, E, H, pad = 2, 300, 8, 16, 7168, 1
+    topk, w, h = make(404, R, S, K, E, H)
+    N = R * S
+    g = gpu_layout(topk, R, S, E, pad)
+    cap = g["dev"]["cap"]
+    base = torch.empty(N * H + 8, dtype=torch.int16, device=DEV)
+    hid = base[8:].view(N, H)
+    hid.copy_(torch.from_numpy(h.view(np.int16)).to(DEV))
+    hid = hid.view(torch.bfloat16)
+    assert hid.data_ptr() % 32 == 16
+    if fp8:
+        rbase = torch.full((cap * H + 16,), RECV_FP8_FILL, dtype=torch.uint8,
+                           device=DEV)
+        recv = rbase[16:].view(cap, H)
+        scales = torch.full((cap, H // 128), SCALE_FILL, dtype=torch.float32,
+                            device=DEV)
+    else:
+        rbase = torch.full((cap * H + 8,), RECV_BF16_FILL, dtype=torch.int16,
+                           device=DEV)
+        recv = rbase[8:].view(cap, H).view(torch.bfloat16)
+        scales = None
+    assert recv.data_ptr() % 32 == 16
+    recv_w = torch.full((cap,), RECV_W_FILL, dtype=torch.float32, device=DEV)
+    st = status_tensor()
+    ep.ep_dispatch(hid, to_dev(w), g["dev"]["pos"], g["dev"]["row_src"],
+                   g["dev"]["offsets"], N, K, E, H, fp8, recv, scales, recv_w,
+                   status=st, cap=cap)
+    torch.cuda.synchronize()
+    assert int(st[0].item()) == 0
+    o_lay = oracle.layout(topk, E, pad, cap)
+    if fp8:
+        r, sc, rw = oracle.dispatch_fp8(h, w, o_lay, E, cap,
+                                        recv_fill=RECV_FP8_FILL,
+                                        scale_fill=SCALE_FILL,
+                                        recv_w_fill=RECV_W_FILL)
+        np.testing.assert_array_equal(recv.cpu().numpy(), r)
+        np.testing.assert_array_equal(scales.cpu().numpy(), sc)
+    else:
+        r, rw = oracle.dispatch_bf16(h, w, o_lay, E, cap,
+                                     recv_fill=RECV_BF16_FILL,
+                                     recv_w_fill=RECV_W_FILL)
+        np.testing.assert_array_equal(u16(recv), r)
+    np.testing.assert_array_equal(recv_w.cpu().numpy(), rw)
 
 
 @pytest.mark.parametrize("fp8", [False, True])
