@@ -176,7 +176,13 @@ EP_API int ep_layout_static(const int32_t* topk_experts, int R, int S, int K,
  *                        ignored (may be NULL)
  *      recv_weights      fp32 [cap]: w[t,k] at pos[t,k], 0 on padding rows;
  *                        may be NULL
- *      num_sms           SMs to use, 0 = all
+ *      num_sms           SMs to use, 0 = all. With all SMs (0, or at least
+ *                        the device's count) the copy runs one CTA per
+ *                        token; with fewer it runs persistent CTAs on that
+ *                        many SMs. The results are the same bits either way.
+ *                        hidden and recv 32-byte aligned (and H % 16 == 0
+ *                        for bf16) let the per-token kernels use 32-byte
+ *                        accesses; 16-byte alignment is enough.
  *      status            EP_DEV_CAPACITY, EP_DEV_TIMEOUT may be OR-ed in
  */
 EP_API int ep_dispatch(const void* hidden, const float* route_weights,
