@@ -12,8 +12,9 @@
 // 1/(K+1) of the bytes they move (bf16) and HBM write bandwidth bounds them.
 // With every SM in use, one CTA per token:
 //
-//   k_dispatch_bf16_tok  each thread loads 16-byte vectors of the row and
-//                        stores each to the K rows.
+//   k_dispatch_bf16_tok  each thread loads 32-byte vectors of the row (16
+//                        bytes when the buffers are only 16-byte aligned)
+//                        and stores each to the K rows.
 //   k_dispatch_fp8_tok   each warp loads two 512-channel units, quantises
 //                        them in registers and stores codes and scales to
 //                        the K rows.
@@ -321,7 +322,8 @@ __global__ void __launch_bounds__((kMaxConsumerWarps + 1) * 32, 2)
 
 // ---------------------------------------------------------------------------
 // bf16, one token per CTA (every SM in use): the threads load the token row
-// with 16-byte loads and store each vector to the K rows. CTAs are short and
+// in 32-byte vectors (kWide: hidden and recv 32-byte aligned, H % 16 == 0;
+// else 16-byte vectors) and store each to the K rows. CTAs are short and
 // the hardware starts them in token order, so the rows being written at any
 // moment belong to a narrow, advancing window of tokens; persistent CTAs
 // drift apart and spread the writes over many more DRAM pages (measured on
@@ -383,7 +385,8 @@ __global__ void __launch_bounds__(kMaxConsumerWarps * 32)
 
 // ---------------------------------------------------------------------------
 // FP8, one token per CTA (every SM in use): each warp loads two 512-channel
-// units of the row with 16-byte loads before it quantises either, then
+// units of the row (a lane's 32 bytes of a unit in one load when kWide:
+// hidden 32-byte aligned) before it quantises either, then
 // quantises each unit in registers (a lane's 16 channels, 8 lanes per
 // 128-channel group, as in the persistent kernel) and stores its 16 codes to
 // the K rows; lanes 8g store the group's scale. 224 threads cover H=7168, so
