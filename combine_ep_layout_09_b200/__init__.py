@@ -9,7 +9,8 @@ from ._binding import (  # noqa: F401
     EP_WAIT_SITE_SMALL, EP_WAIT_SITE_TILE_REDUCE, EP_ERR_CAPACITY, EP_ERR_CUDA,
     EP_ERR_INVALID_ARG, EP_ERR_WORKSPACE, EP_OK, EPError, ep_abi_version,
     ep_capacity_bound, ep_combine, ep_combine_backward, ep_combine_recv_weights, ep_debug_bounded_wait,
-    ep_debug_e4m3_encode, ep_debug_force_timeouts, ep_debug_quantize, ep_dispatch,
+    ep_debug_e4m3_encode, ep_debug_force_timeouts, ep_debug_quantize,
+    ep_debug_stream_read, ep_dispatch,
     ep_dispatch_backward, ep_gather_route_weights, ep_layout, ep_layout_dispatch,
     ep_layout_workspace_bytes,
     ep_plan_balanced, ep_prefetch_weights, ep_reduce_slot_grads, ep_strerror, lib, library_path,

@@ -119,6 +119,8 @@ def _declare(L):
     L.ep_debug_quantize.argtypes = [P, P, P, i64, P]
     L.ep_debug_bounded_wait.restype = i32
     L.ep_debug_bounded_wait.argtypes = [P, i64, P, P]
+    L.ep_debug_stream_read.restype = i32
+    L.ep_debug_stream_read.argtypes = [P, i64, P, P]
     L.ep_debug_force_timeouts.restype = i32
     L.ep_debug_force_timeouts.argtypes = [ctypes.c_uint32, i64]
 
@@ -416,6 +418,18 @@ def ep_debug_bounded_wait(flag, max_polls, status, stream=None):
         _ptr(flag, "flag", _I32, 1), int(max_polls),
         _ptr(status, "status", _I32, 1), _stream(stream))
     _check(rc, "ep_debug_bounded_wait")
+
+
+def ep_debug_stream_read(src, sink, stream=None):
+    """Read all of `src` (a CUDA tensor, 32-byte aligned, a multiple of 32
+    bytes) once; the XOR of its 32-bit words is XOR-ed into sink[0]."""
+    nbytes = src.numel() * src.element_size()
+    if not src.is_cuda or not src.is_contiguous():
+        raise ValueError("src must be a contiguous CUDA tensor")
+    rc = lib().ep_debug_stream_read(
+        ctypes.c_void_p(src.data_ptr()), int(nbytes),
+        _ptr(sink, "sink", (torch.int32,), 1), _stream(stream))
+    _check(rc, "ep_debug_stream_read")
 
 
 def ep_debug_force_timeouts(sites, budget_ns=0):

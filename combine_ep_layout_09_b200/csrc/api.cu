@@ -8,7 +8,7 @@
 
 namespace {
 
-constexpr int kAbiVersion = 4;  // 4: ep_combine_recv_weights, ep_debug_force_timeouts, prefetch status
+constexpr int kAbiVersion = 5;  // 5: ep_debug_stream_read
 constexpr int kMaxK = 32;
 constexpr int kMaxH = 32768;
 constexpr int64_t kMaxEntries = (int64_t(1) << 30) - 1;
@@ -359,6 +359,16 @@ int ep_debug_bounded_wait(const int32_t* flag, int64_t max_polls,
   if (!aligned16(flag) || status == nullptr || !status_ok(status))
     return EP_ERR_ALIGNMENT;
   return cuda_rc(ep::launch_debug_wait(flag, max_polls, status, as_stream(stream)));
+}
+
+int ep_debug_stream_read(const void* src, int64_t bytes, uint32_t* sink,
+                         void* stream) {
+  if (bytes < 0 || bytes % 32 != 0 || sink == nullptr) return EP_ERR_INVALID_ARG;
+  if (bytes == 0) return EP_OK;
+  if ((reinterpret_cast<uintptr_t>(src) & 31u) != 0 ||
+      (reinterpret_cast<uintptr_t>(sink) & 3u) != 0)
+    return EP_ERR_ALIGNMENT;
+  return cuda_rc(ep::launch_debug_stream_read(src, bytes, sink, as_stream(stream)));
 }
 
 int ep_debug_force_timeouts(uint32_t sites, int64_t budget_ns) {

@@ -13,7 +13,7 @@
 //                  warp bulk-loads the K gathered part-rows of a (token, part)
 //                  unit into a shared-memory stage (three stages, ~170 KB of
 //                  reads in flight per SM); consumer threads reduce from
-//                  shared memory; one thread bulk-stores the output part.
+//                  shared memory and store the output part from registers.
 //   k_combine<K>   (small batches) CTAs walk tokens, threads split the row
 //                  into 16-byte vectors and issue their K gathered loads
 //                  before any arithmetic.
@@ -144,13 +144,12 @@ __global__ void __launch_bounds__(kCombineMaxThreads, 2)
 // ---------------------------------------------------------------------------
 // TMA-fed combine: a producer warp bulk-loads, for each (token, row part),
 // the K gathered part-rows into a shared-memory stage; consumer threads run
-// the fma chain from shared memory and one thread bulk-stores the output
-// part. Three stages keep ~170 KB of reads in flight per SM.
+// the fma chain from shared memory and store their 16-byte output vectors
+// from registers. Three stages keep ~170 KB of reads in flight per SM.
 // ---------------------------------------------------------------------------
 
 constexpr int kTmaMaxConsumerWarps = 16;
 constexpr int kTmaStages = 3;
-constexpr int kTmaOutStages = 2;
 constexpr uint32_t kTmaStageTarget = 64 * 1024;  // K part-rows per stage
 
 __host__ __device__ constexpr uint32_t al128(uint32_t x) { return (x + 127u) & ~127u; }
@@ -159,7 +158,7 @@ struct TmaShape {
   int part_ch;   // channels per part (multiple of 8)
   int parts;     // parts per row
   int cw;        // consumer warps
-  uint32_t in_bytes, out_bytes;
+  uint32_t in_bytes;
   size_t smem;
 };
 
@@ -173,10 +172,8 @@ __host__ __device__ inline TmaShape tma_shape(int H, int K) {
   int cw = (part_v + 31) / 32;
   sh.cw = cw < kTmaMaxConsumerWarps ? cw : kTmaMaxConsumerWarps;
   sh.in_bytes = al128(uint32_t(K) * uint32_t(sh.part_ch) * 2u);
-  sh.out_bytes = al128(uint32_t(sh.part_ch) * 2u);
-  // stages, output stages, then per stage: full / empty barriers, mask, weights
-  sh.smem = size_t(kTmaStages) * sh.in_bytes + size_t(kTmaOutStages) * sh.out_bytes +
-            size_t(kTmaStages) * (16 + 4 + 4 * 32) + 64;
+  // stages, then per stage: full / empty barriers, mask, weights
+  sh.smem = size_t(kTmaStages) * sh.in_bytes + size_t(kTmaStages) * (16 + 4 + 4 * 32) + 64;
   return sh;
 }
 
@@ -189,8 +186,7 @@ __global__ void __launch_bounds__((kTmaMaxConsumerWarps + 1) * 32, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cw = sh.cw;
   uint8_t* in_base = smem;
-  uint8_t* out_base = smem + size_t(kTmaStages) * sh.in_bytes;
-  uint8_t* meta = out_base + size_t(kTmaOutStages) * sh.out_bytes;
+  uint8_t* meta = smem + size_t(kTmaStages) * sh.in_bytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(meta);
   uint64_t* empty = full + kTmaStages;
   uint32_t* vmask = reinterpret_cast<uint32_t*>(empty + kTmaStages);
@@ -276,8 +272,8 @@ __global__ void __launch_bounds__((kTmaMaxConsumerWarps + 1) * 32, 1)
       }
     __syncwarp();
   } else {
-    // ---- consumers --------------------------------------------------------
-    const bool issuer = (warp == 0 && lane == 0);
+    // ---- consumers: each warp follows the stages on its own and stores its
+    // threads' 16-byte output vectors from registers ------------------------
     const int nthreads = cw * 32;
     int it = 0;
     for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++it) {
@@ -287,11 +283,15 @@ __global__ void __launch_bounds__((kTmaMaxConsumerWarps + 1) * 32, 1)
       const int len = min(sh.part_ch, H - c0);
       const int s = it % kTmaStages;
       const uint32_t ph = uint32_t(it / kTmaStages) & 1u;
-      uint8_t* ob = out_base + size_t(it % kTmaOutStages) * sh.out_bytes;
       bool ok = true;
       if (lane == 0) ok = mbar_wait_bounded(&full[s], ph, forced);
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok && lane == 0) report(status, EP_DEV_TIMEOUT);
+      if (!ok) {
+        // the producer has stopped or the wait was forced: leave without
+        // touching the stage (its producer waits on `empty` time out too)
+        if (lane == 0) report(status, EP_DEV_TIMEOUT);
+        break;
+      }
       const uint32_t m = vmask[s];
       const uint8_t* st = in_base + size_t(s) * sh.in_bytes;
       for (int v = threadIdx.x; v < (len >> 3); v += nthreads) {
@@ -302,21 +302,11 @@ __global__ void __launch_bounds__((kTmaMaxConsumerWarps + 1) * 32, 1)
                                                           size_t(v) * 16);
           fma8(acc, wk[s * 32 + k], d);
         }
-        *reinterpret_cast<uint4*>(ob + size_t(v) * 16) = pack8(acc);
+        st_v4(out + t * H + c0 + v * 8, pack8(acc));
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
-      fence_proxy_async_smem();
-      // the other output stage must have been read by its store
-      if (issuer) bulk_wait_read<0>();
-      // every consumer warp leaves together once any of them gave up
-      if (named_barrier_or(1, nthreads, !ok)) break;
-      if (issuer) {
-        bulk_s2g(out + t * H + c0, ob, uint32_t(len) * 2u);
-        bulk_commit();
-      }
     }
-    if (issuer) bulk_wait_all<0>();
   }
 }
 

@@ -107,6 +107,8 @@ cudaError_t launch_debug_quantize(const float* x, const float* scale,
                                   uint8_t* out, int64_t n, cudaStream_t stream);
 cudaError_t launch_debug_wait(const int32_t* flag, int64_t max_polls,
                               int32_t* status, cudaStream_t stream);
+cudaError_t launch_debug_stream_read(const void* src, int64_t bytes,
+                                     uint32_t* sink, cudaStream_t stream);
 
 // Forced give-ups of the listed wait sites (EP_WAIT_SITE_* bits) on the
 // current device, one setter per translation unit that holds wait sites.

@@ -387,6 +387,24 @@ __global__ void k_debug_wait(const int32_t* flag, int64_t max_polls,
   report(status, EP_DEV_TIMEOUT);
 }
 
+// Streaming read of `bytes` bytes (a multiple of 32, 32-byte aligned) with
+// 256-bit loads from every thread; the XOR of all 32-bit words goes to
+// *sink so that nothing can be skipped.
+__global__ void __launch_bounds__(512)
+    k_debug_stream_read(const uint8_t* __restrict__ src, int64_t bytes,
+                        uint32_t* __restrict__ sink) {
+  uint32_t acc = 0;
+  for (int64_t i = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) * 32; i < bytes;
+       i += int64_t(gridDim.x) * blockDim.x * 32) {
+    uint4 lo, hi;
+    ld_stream_v8(src + i, lo, hi);
+    acc ^= lo.x ^ lo.y ^ lo.z ^ lo.w ^ hi.x ^ hi.y ^ hi.z ^ hi.w;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc ^= __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) atomicXor(sink, acc);
+}
+
 }  // namespace
 
 cudaError_t launch_plan_balanced(const int32_t* counts, int R, int S, int K,
@@ -475,6 +493,17 @@ cudaError_t launch_debug_e4m3(const float* x, uint8_t* out, int64_t n,
 cudaError_t launch_debug_wait(const int32_t* flag, int64_t max_polls,
                               int32_t* status, cudaStream_t stream) {
   k_debug_wait<<<1, 32, 0, stream>>>(flag, max_polls, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_debug_stream_read(const void* src, int64_t bytes,
+                                     uint32_t* sink, cudaStream_t stream) {
+  if (bytes == 0) return cudaSuccess;
+  // four 512-thread CTAs per SM: the fastest of 1, 2 and 4 in a probe
+  const int64_t grid = std::max<int64_t>(
+      1, std::min<int64_t>(int64_t(device_sm_count()) * 4, (bytes + 16383) / 16384));
+  k_debug_stream_read<<<int(grid), 512, 0, stream>>>(
+      static_cast<const uint8_t*>(src), bytes, sink);
   return cudaGetLastError();
 }
 

@@ -434,6 +434,14 @@ EP_API int ep_debug_quantize(const float* x, const float* group_scale,
 EP_API int ep_debug_bounded_wait(const int32_t* flag, int64_t max_polls,
                           int32_t* status, void* stream);
 
+/* Read `bytes` bytes at src (32-byte aligned, bytes % 32 == 0) once with
+ * 256-bit loads from four 512-thread CTAs per SM, and XOR every 32-bit word
+ * into *sink (caller-zeroed, 4-byte aligned). A measuring stick for the
+ * read side of the roofline: on the B200 it streams 4 GiB faster than a
+ * framework reduction does. */
+EP_API int ep_debug_stream_read(const void* src, int64_t bytes, uint32_t* sink,
+                                void* stream);
+
 /* Wait sites of the shipped kernels, for ep_debug_force_timeouts. */
 #define EP_WAIT_SITE_LOOKBACK 1u    /* layout, two-kernel path: look-back over
                                        the earlier tiles' published counts */

@@ -41,7 +41,7 @@ def test_library_is_the_in_tree_build():
 
 
 def test_pure_host_entry_points():
-    assert ep.ep_abi_version() == 4
+    assert ep.ep_abi_version() == 5
     assert ep.ep_capacity_bound(32768, 8, 256, 128) == 32768 * 8 + 256 * 127
     assert ep.ep_capacity_bound(10, 2, 4, 1) == 20
     assert ep.ep_capacity_bound(-1, 2, 4, 1) < 0
@@ -164,6 +164,19 @@ def test_force_timeouts_rejects_on_host():
         ep.EP_ERR_INVALID_ARG
     assert lib.ep_debug_force_timeouts(ep.EP_WAIT_SITE_DISPATCH,
                                        3_000_000_000) == ep.EP_ERR_INVALID_ARG
+
+
+def test_stream_read_rejects_on_host():
+    lib = _raw()
+    P = ctypes.c_void_p
+    lib.ep_debug_stream_read.argtypes = [P, ctypes.c_int64, P, P]
+    ok = P(1 << 20)                       # aligned; never dereferenced
+    assert lib.ep_debug_stream_read(ok, 33, ok, None) == ep.EP_ERR_INVALID_ARG
+    assert lib.ep_debug_stream_read(ok, -32, ok, None) == ep.EP_ERR_INVALID_ARG
+    assert lib.ep_debug_stream_read(ok, 64, None, None) == ep.EP_ERR_INVALID_ARG
+    assert lib.ep_debug_stream_read(P((1 << 20) + 16), 64, ok, None) == \
+        ep.EP_ERR_ALIGNMENT
+    assert lib.ep_debug_stream_read(ok, 0, ok, None) == ep.EP_OK
 
 
 def test_binding_rejects_host_tensors():

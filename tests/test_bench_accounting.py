@@ -76,7 +76,9 @@ def _combine_constants():
     (1024, 8, 7168, "k_combine<8>"),      # decode: 2048 units < 16 per SM
     (2500, 8, 1024, "k_combine_tma"),     # one part, 2500 units
     (300, 8, 7168, "k_combine<8>"),
-    (100000, 1, 32768, "k_combine<1>"),   # 64 KB parts: stages above 200 KB
+    (100000, 1, 32768, "k_combine_tma"),  # one 64 KB part: 192 KB of stages
+    (100000, 2, 32768, "k_combine_tma"),  # two 64 KB parts
+    (2000, 1, 32768, "k_combine<1>"),     # 2000 units < 16 per SM
 ])
 def test_combine_kernel_follows_the_library_rule(N, K, H, expect):
     assert _combine_constants() == (64, 200, 16)   # what bench.py mirrors

@@ -84,6 +84,7 @@ def test_k_order_and_fma_cases():
     (2500, 8, 7176, 4000),    # two parts per row, the last one shorter
     (5000, 3, 520, 6000),     # one part per row
     (2400, 32, 2056, 9000),   # K=32: three parts of 688 / 688 / 680 channels
+    (2400, 1, 32768, 2600),   # K=1, the widest row: one 64 KB part per stage
 ])
 def test_large_batches_tma_path(N, K, H, rows):
     # enough (token, part) units per SM that the bulk-copy pipeline runs
