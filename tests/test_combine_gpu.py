@@ -86,7 +86,9 @@ def test_k_order_and_fma_cases():
     (2400, 32, 2056, 9000),   # K=32: three parts of 688 / 688 / 680 channels
     (2400, 1, 32768, 2600),   # K=1, the widest row: one 64 KB part per stage
 ])
-def test_large_batches_tma_path(N, K, H, rows):
+# the persistent pipeline on every SM (0) and on fewer (100)
+@pytest.mark.parametrize("num_sms", [0, 100])
+def test_large_batches_tma_path(N, K, H, rows, num_sms):
     # enough (token, part) units per SM that the bulk-copy pipeline runs
     rng = np.random.default_rng(N + K)
     y = u16(workloads.bf16_normal((rows, H), K))
@@ -94,7 +96,7 @@ def test_large_batches_tma_path(N, K, H, rows):
     pos[rng.random(pos.shape) < 0.05] = -1
     pos[7] = -1                                  # a token with no rows
     w = rng.standard_normal((N, K)).astype(np.float32)
-    got = check(y, pos, w)
+    got = check(y, pos, w, num_sms=num_sms)
     assert np.all(got[7] == 0)
 
 
@@ -116,7 +118,8 @@ def test_widest_row_and_k32():
     (2500, 8, 1024, 9000),    # bulk-copy pipeline
     (2400, 8, 7176, 4000),    # bulk-copy pipeline, two parts per row
 ])
-def test_receive_side_weights(N, K, H, rows):
+@pytest.mark.parametrize("num_sms", [0, 100])
+def test_receive_side_weights(N, K, H, rows, num_sms):
     # weight of (t,k) = recv_weights[pos[t,k]], handed back in token order
     rng = np.random.default_rng(N * K + H)
     y = u16(workloads.bf16_normal((rows, H), N + 7))
@@ -129,12 +132,12 @@ def test_receive_side_weights(N, K, H, rows):
     gathered = torch.full((N, K), -7.0, dtype=torch.float32, device="cuda:0")
     st = torch.zeros(4, dtype=torch.int32, device="cuda:0")
     ep.ep_combine_recv_weights(to_bf16_dev(y), to_dev(pos), to_dev(rw), N, K,
-                               H, out, gathered, status=st)
+                               H, out, gathered, num_sms=num_sms, status=st)
     assert int(st[0].item()) == 0
     np.testing.assert_array_equal(gathered.cpu().numpy(), gw_ref)
     np.testing.assert_array_equal(u16(out), oracle.combine(y, pos, gw_ref))
     # without the gathered output: the same result
     out2 = torch.empty_like(out)
     ep.ep_combine_recv_weights(to_bf16_dev(y), to_dev(pos), to_dev(rw), N, K,
-                               H, out2, None)
+                               H, out2, None, num_sms=num_sms)
     assert torch.equal(out2.view(torch.int16), out.view(torch.int16))

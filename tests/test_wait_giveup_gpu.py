@@ -239,8 +239,10 @@ def test_small_batch_waits_give_up(fp8, num_sms):
     check_dispatch(recv, scales, recv_w, topk, w, h, E, pad, cap, fp8)
 
 
-def test_combine_waits_give_up():
-    # enough (token, part) units per SM for the bulk-copy pipeline
+# the persistent pipeline on every SM (0) and on fewer (100)
+@pytest.mark.parametrize("num_sms", [0, 100])
+def test_combine_waits_give_up(num_sms):
+    # enough (token, part) units per SM for the bulk-copy kernels
     N, K, H, rows = 2500, 8, 1024, 9000
     rng = np.random.default_rng(8)
     y = u16(workloads.bf16_normal((rows, H), 9))
@@ -252,7 +254,7 @@ def test_combine_waits_give_up():
         out = torch.full((N + GUARD, H), RECV_BF16_FILL, dtype=torch.int16,
                          device=DEV).view(torch.bfloat16)
         st = status_tensor()
-        ep.ep_combine(yd, pd, wd, N, K, H, out, status=st)
+        ep.ep_combine(yd, pd, wd, N, K, H, out, num_sms=num_sms, status=st)
         torch.cuda.synchronize()
         return out, int(st[0].item())
 
