@@ -90,7 +90,7 @@ __host__ __device__ inline SmallPlan small_plan(int64_t N, int K, int E, int H,
   return p;
 }
 
-// Bounded wait of lane 0 on `bar`, the verdict shared by the warp.
+// Bounded wait of lane 0 on `bar`, the outcome shared by the warp.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity,
                                           int32_t* status, bool forced) {
   bool ok = true;
